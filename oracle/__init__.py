@@ -1,0 +1,162 @@
+"""CPU oracle for SubMConv3d -- TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline leg
+may import this package.  The product path (the CUDA library and its binding)
+never imports or calls it, and it imports nothing from the product path.
+
+Two independent implementations of the same definition:
+
+* ``neighbor_map`` / ``forward``: plain C (``subm_oracle.c``), fp64, a sorted-key
+  dictionary searched with ``bsearch`` and a per-voxel loop over offsets.
+* ``neighbor_map_py`` / ``forward_py``: pure Python with a ``dict`` and loops,
+  for tiny inputs only.
+
+The definition (lato.2_mrp_mlx README, "Status" and "Correctness" sections;
+pixal3d_mrp_mlx README, "Status", for the [K^3, in, out] weight layout):
+
+    out[i] = bias + sum_{d in {-1,0,1}^3, p_i + d active} W[k(d)]^T x[index(p_i + d)]
+
+with the offset order k(d) = (dx+1)*9 + (dy+1)*3 + (dz+1) (a reading: the
+pages do not fix it), cross-correlation orientation (gather p + d), batch
+isolation, and grid-boundary neighbours treated as holes.
+
+Pins: every function here is pinned by ``tests/test_oracle_pins.py`` against
+dense brute force, torch's CPU conv3d, closed forms and invariants; none is
+"parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "subm_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+
+OK, INVALID_ARG, COORD_RANGE, DUPLICATE, OOM = 0, 1, 3, 4, 6
+
+
+class OracleError(RuntimeError):
+    def __init__(self, code: int):
+        super().__init__(f"oracle error code {code}")
+        self.code = code
+
+
+def build(force: bool = False) -> str:
+    """Compile subm_oracle.c into liboracle.so with gcc (plain -O2, no fast-math)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-o", tmp, _SRC])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        lib.oracle_neighbor_map.restype = ctypes.c_int
+        lib.oracle_neighbor_map.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                            ctypes.c_int32, ctypes.c_void_p]
+        lib.oracle_forward_f64.restype = ctypes.c_int
+        lib.oracle_forward_f64.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32,
+                                           ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
+                                           ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
+                                           ctypes.c_int64, ctypes.c_void_p]
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray | None) -> int | None:
+    return None if a is None else a.ctypes.data
+
+
+def neighbor_map(coords: np.ndarray, extent, kernel_size: int = 3) -> np.ndarray:
+    """int32 [N, K^3]: row index of the active voxel at p_i + d_k, or -1."""
+    coords = np.ascontiguousarray(coords, dtype=np.int32).reshape(-1, 4)
+    ext = np.ascontiguousarray(extent, dtype=np.int32).reshape(3)
+    kvol = kernel_size ** 3
+    nbr = np.empty((coords.shape[0], kvol), dtype=np.int32)
+    rc = _load().oracle_neighbor_map(_ptr(coords), coords.shape[0], _ptr(ext), kernel_size, _ptr(nbr))
+    if rc != OK:
+        raise OracleError(rc)
+    return nbr
+
+
+def forward(nbr: np.ndarray, x: np.ndarray, w: np.ndarray, bias: np.ndarray | None = None,
+            rows: np.ndarray | None = None) -> np.ndarray:
+    """fp64 output rows ``rows`` (all rows when None) of the convolution over ``nbr``."""
+    nbr = np.ascontiguousarray(nbr, dtype=np.int32)
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    w = np.ascontiguousarray(w, dtype=np.float64)
+    kvol, cin, cout = w.shape
+    n = x.shape[0]
+    assert nbr.shape == (n, kvol) and x.shape[1] == cin
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float64).reshape(cout)
+    r = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64).reshape(-1)
+    nrows = n if r is None else r.shape[0]
+    out = np.empty((nrows, cout), dtype=np.float64)
+    rc = _load().oracle_forward_f64(_ptr(nbr), n, kvol, _ptr(x), cin, _ptr(w), _ptr(b), cout,
+                                    _ptr(r), nrows, _ptr(out))
+    if rc != OK:
+        raise OracleError(rc)
+    return out
+
+
+def subm_conv3d(coords, extent, x, w, bias=None, rows=None):
+    """Convenience: neighbour map then forward (kernel size from w.shape[0])."""
+    ks = {1: 1, 27: 3}[int(np.shape(w)[0])]
+    return forward(neighbor_map(coords, extent, ks), x, w, bias, rows)
+
+
+# ---------------------------------------------------------------------------
+# Pure-Python twin (dict lookup, per-voxel loop) for tiny inputs.
+# ---------------------------------------------------------------------------
+
+def _offsets(kernel_size: int):
+    r = kernel_size // 2
+    return [(dx, dy, dz) for dx in range(-r, r + 1) for dy in range(-r, r + 1) for dz in range(-r, r + 1)]
+
+
+def neighbor_map_py(coords, extent, kernel_size: int = 3) -> np.ndarray:
+    coords = np.asarray(coords).reshape(-1, 4).tolist()
+    ex, ey, ez = (int(v) for v in extent)
+    table = {}
+    for i, (b, x, y, z) in enumerate(coords):
+        if not (0 <= b <= 65535 and 0 <= x < ex and 0 <= y < ey and 0 <= z < ez):
+            raise OracleError(COORD_RANGE)
+        if (b, x, y, z) in table:
+            raise OracleError(DUPLICATE)
+        table[(b, x, y, z)] = i
+    offs = _offsets(kernel_size)
+    nbr = np.full((len(coords), len(offs)), -1, dtype=np.int32)
+    for i, (b, x, y, z) in enumerate(coords):
+        for k, (dx, dy, dz) in enumerate(offs):
+            nbr[i, k] = table.get((b, x + dx, y + dy, z + dz), -1)
+    return nbr
+
+
+def forward_py(nbr, x, w, bias=None) -> np.ndarray:
+    nbr = np.asarray(nbr)
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    kvol, cin, cout = w.shape
+    out = np.zeros((x.shape[0], cout), dtype=np.float64)
+    for i in range(x.shape[0]):
+        acc = [0.0] * cout if bias is None else [float(v) for v in np.asarray(bias, dtype=np.float64)]
+        for k in range(kvol):
+            j = int(nbr[i, k])
+            if j < 0:
+                continue
+            for ci in range(cin):
+                xv = float(x[j, ci])
+                for co in range(cout):
+                    acc[co] += xv * float(w[k, ci, co])
+        out[i] = acc
+    return out
