@@ -1,0 +1,162 @@
+/*
+ * spconv.h -- C ABI of the B200 (sm_100a) submanifold sparse 3-D convolution
+ * library (SubMConv3d, kernel size 3 or 1, stride 1).
+ *
+ * The operation (lato.2_mrp_mlx README, sections "The scope, once measured",
+ * "Status" and "Correctness"; pixal3d_mrp_mlx README, "Status", for the weight
+ * layout):
+ *
+ *   out[i] = bias + sum over d in {-1,0,1}^3 with p_i + d active of
+ *            W[k(d)]^T x[index of p_i + d]
+ *
+ * Outputs exist only at the input's active voxels (stride 1, no padding), the
+ * neighbour is gathered at p + d (cross-correlation), a neighbour must share the
+ * batch index, and neighbours outside [0, extent) are holes.  The offset order
+ * is k(d) = (dx+1)*9 + (dy+1)*3 + (dz+1), dx slowest (x, y, z = coordinate
+ * columns 1, 2, 3); the centre offset is k = 13.
+ *
+ * The neighbour map is built once per coordinate set and cached in a handle,
+ * as the pages' "cached device index" does (lato.2_mrp_mlx README, "Fleet
+ * benchmark"); the map build is the step the same section names as dominant
+ * whenever coordinates change.  The trellis-mac article (section on sparse 3D
+ * convolution, gather-scatter) builds a hash map of active voxel coordinates
+ * first and probes it per kernel offset; the build here does the same on the GPU.
+ *
+ * Conventions for every call:
+ *   - Pointers documented as "device" must point to memory of the current CUDA
+ *     device, 16-byte aligned.  Pointers documented as "host" are host memory.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream).
+ *   - The caller owns every buffer it passes; the library keeps no pointer to a
+ *     caller buffer after a call returns.
+ *   - Errors are returned as spconv_status_t; nothing aborts or throws across
+ *     the ABI.  spconv_last_error() gives a message for the calling thread's
+ *     most recent failure.
+ */
+#ifndef SPCONV_B200_H
+#define SPCONV_B200_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SPCONV_API __attribute__((visibility("default")))
+#else
+#define SPCONV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct spconv_map_s* spconv_map_t; /* opaque, owned by the library */
+
+typedef enum {
+    SPCONV_OK = 0,
+    SPCONV_ERR_INVALID_ARG = 1,  /* null pointer, bad size, bad alignment, bad extent */
+    SPCONV_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. bf16 with C % 16 != 0) */
+    SPCONV_ERR_COORD_RANGE = 3,  /* a coordinate outside [0, extent) or batch outside [0, 65535] */
+    SPCONV_ERR_DUPLICATE = 4,    /* the same (b, x, y, z) appears twice */
+    SPCONV_ERR_TABLE_FULL = 5,   /* the hash table ran out of slots */
+    SPCONV_ERR_OOM = 6,          /* a device allocation failed */
+    SPCONV_ERR_CUDA = 7,         /* a CUDA runtime call failed */
+    SPCONV_ERR_TIMEOUT = 8       /* a bounded device-side wait gave up */
+} spconv_status_t;
+
+typedef enum { SPCONV_F32 = 0, SPCONV_BF16 = 1 } spconv_dtype_t;
+
+/*
+ * Build the neighbour map of a coordinate set.
+ *
+ *   coords       device int32 [n, 4], row-major, columns (b, x, y, z).
+ *   n            number of active voxels, 0 <= n < 2^31.  n = 0 gives an empty map.
+ *   extent       host int32 [3] = (X, Y, Z), each in [1, 65535].
+ *   kernel_size  3 (27 offsets) or 1 (the map is the identity and is not stored).
+ *   stream       stream on which the build runs.
+ *   out_map      receives the handle on success; untouched on failure.
+ *
+ * Device work: pack (b, x, y, z) into a 64-bit key and validate it; insert the
+ * keys into an open-addressing hash table (linear probing, 64-bit CAS, load
+ * factor <= 1/2); probe the 27 offsets of every voxel and write the dense map
+ * nbr[i*27 + k] = row of p_i + d_k, or -1.  The call synchronises `stream`
+ * once, to read the device error flags, and returns only a valid map.
+ * Errors: SPCONV_ERR_COORD_RANGE, SPCONV_ERR_DUPLICATE, SPCONV_ERR_TABLE_FULL,
+ * SPCONV_ERR_INVALID_ARG, SPCONV_ERR_OOM, SPCONV_ERR_CUDA.
+ * The map may be used on any stream of the same device after the call returns.
+ */
+SPCONV_API spconv_status_t spconv_build_map(const int32_t* coords, int64_t n, const int32_t* extent,
+                                 int32_t kernel_size, void* stream, spconv_map_t* out_map);
+
+/*
+ * Run one SubMConv3d layer over a map.
+ *
+ *   map     handle from spconv_build_map.
+ *   dtype   element type shared by x, w, bias and out (SPCONV_F32 or SPCONV_BF16).
+ *   x       device [n, cin] row-major, row i = voxel i of the map's coordinates.
+ *   cin     input channels (bf16: a multiple of 16).
+ *   w       device [K^3, cin, cout] row-major (K^3 = 27 or 1), offset order above.
+ *   bias    device [cout] or NULL (no bias).
+ *   out     device [n, cout] row-major; must not overlap x.  Each row is written once.
+ *   cout    output channels (bf16: a multiple of 16).
+ *   stream  stream on which the layer runs.
+ *
+ * Accumulation is fp32 in every mode; the bf16 result is rounded to nearest even.
+ * The call only validates on the host and launches; it never synchronises.
+ * Errors: SPCONV_ERR_INVALID_ARG, SPCONV_ERR_UNSUPPORTED, SPCONV_ERR_CUDA.  A
+ * device-side wait that gives up is recorded in the map and reported by
+ * spconv_map_check().
+ */
+SPCONV_API spconv_status_t spconv_subm_forward(spconv_map_t map, spconv_dtype_t dtype, const void* x, int32_t cin,
+                                    const void* w, const void* bias, void* out, int32_t cout,
+                                    void* stream);
+
+/* Release a map and its device memory (synchronous with respect to the device).
+ * NULL is accepted and ignored. */
+SPCONV_API spconv_status_t spconv_free(spconv_map_t map);
+
+/*
+ * Introspection of a map (for tests and the benchmark).
+ *   n            receives the voxel count (may be NULL).
+ *   kernel_size  receives 3 or 1 (may be NULL).
+ *   pairs        receives the number of (voxel, offset) pairs with an active
+ *                neighbour, the centre included (n for kernel size 1) (may be NULL).
+ *   nbr_dev      receives the device pointer of the dense int32 [n, 27] map, or
+ *                NULL for kernel size 1 or n = 0 (may be NULL).  The library owns it.
+ */
+SPCONV_API spconv_status_t spconv_map_info(spconv_map_t map, int64_t* n, int32_t* kernel_size, int64_t* pairs,
+                                const int32_t** nbr_dev);
+
+/*
+ * Synchronise `stream` and report (then clear) any device-side wait of a forward
+ * kernel on this map that gave up: SPCONV_OK or SPCONV_ERR_TIMEOUT.
+ */
+SPCONV_API spconv_status_t spconv_map_check(spconv_map_t map, void* stream);
+
+/* Message for the calling thread's most recent failure ("" if none). */
+SPCONV_API const char* spconv_last_error(void);
+
+/*
+ * Forward with an explicit kernel family, for cross-checks:
+ *   SPCONV_ALGO_AUTO     what spconv_subm_forward uses: the tcgen05 kernel for bf16
+ *                        when cout % 64 == 0, the CUDA-core kernel otherwise.
+ *   SPCONV_ALGO_SIMT     CUDA-core FMA kernel, any channel count, fp32 or bf16.
+ *   SPCONV_ALGO_TCGEN05  tcgen05 tensor-core kernel (bf16, cin % 16 == 0,
+ *                        cout % 64 == 0; SPCONV_ERR_UNSUPPORTED otherwise).
+ * Same arguments, ownership and errors as spconv_subm_forward.
+ */
+typedef enum { SPCONV_ALGO_AUTO = 0, SPCONV_ALGO_SIMT = 1, SPCONV_ALGO_TCGEN05 = 2 } spconv_algo_t;
+SPCONV_API spconv_status_t spconv_subm_forward_algo(spconv_map_t map, spconv_dtype_t dtype, const void* x, int32_t cin,
+                                         const void* w, const void* bias, void* out, int32_t cout,
+                                         spconv_algo_t algo, void* stream);
+
+/*
+ * Test hook: force the hash-table slot count of later builds in this process
+ * (0 restores the automatic choice, a power of two >= 2n).  Lets a test reach
+ * SPCONV_ERR_TABLE_FULL with a small table.  `slots` must be 0 or a power of two.
+ */
+SPCONV_API spconv_status_t spconv_debug_set_table_slots(int64_t slots);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPCONV_B200_H */

@@ -1,0 +1,163 @@
+"""Python binding of the B200 SubMConv3d library (``include/spconv.h``).
+
+Argument marshalling only: every step of the hot path (map build, gather, GEMM,
+store) runs in the CUDA library ``libspconv_b200.so``.  PyTorch supplies device
+memory and the current stream.  Importing this package fails loudly if the
+library has not been built (``python -m submanifold_sparse_convolution_submconv3d_b200.build``).
+
+The functions carry the C names:
+
+* ``spconv_build_map(coords, extent, kernel_size=3)`` -> ``SubmMap``
+* ``spconv_subm_forward(map, x, w, bias=None, out=None)`` -> ``out``
+* ``spconv_free(map)``
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libspconv_b200.so")
+
+OK, INVALID_ARG, UNSUPPORTED, COORD_RANGE, DUPLICATE, TABLE_FULL, OOM, CUDA_ERROR, TIMEOUT = range(9)
+ALGO_AUTO, ALGO_SIMT, ALGO_TCGEN05 = 0, 1, 2
+_DTYPES = {torch.float32: 0, torch.bfloat16: 1}
+
+EXPORTED = ("spconv_build_map", "spconv_subm_forward", "spconv_free", "spconv_map_info", "spconv_map_check",
+            "spconv_last_error", "spconv_subm_forward_algo", "spconv_debug_set_table_slots")
+
+
+class SpconvError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"spconv status {status}: {message}")
+        self.status = status
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"CUDA library not built: {LIB_PATH} is missing "
+                          "(run python -m submanifold_sparse_convolution_submconv3d_b200.build)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    lib.spconv_build_map.argtypes = [vp, i64, vp, i32, vp, ctypes.POINTER(vp)]
+    lib.spconv_subm_forward.argtypes = [vp, ctypes.c_int, vp, i32, vp, vp, vp, i32, vp]
+    lib.spconv_subm_forward_algo.argtypes = [vp, ctypes.c_int, vp, i32, vp, vp, vp, i32, ctypes.c_int, vp]
+    lib.spconv_free.argtypes = [vp]
+    lib.spconv_map_info.argtypes = [vp, ctypes.POINTER(i64), ctypes.POINTER(i32), ctypes.POINTER(i64),
+                                    ctypes.POINTER(vp)]
+    lib.spconv_map_check.argtypes = [vp, vp]
+    lib.spconv_debug_set_table_slots.argtypes = [i64]
+    lib.spconv_last_error.restype = ctypes.c_char_p
+    for name in ("spconv_build_map", "spconv_subm_forward", "spconv_subm_forward_algo", "spconv_free",
+                 "spconv_map_info", "spconv_map_check", "spconv_debug_set_table_slots"):
+        getattr(lib, name).restype = ctypes.c_int
+    return lib
+
+
+lib = _load()
+
+
+def _check(status: int) -> None:
+    if status != OK:
+        raise SpconvError(status, lib.spconv_last_error().decode())
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+class SubmMap:
+    """Owns a neighbour-map handle; freed by ``free()`` or garbage collection."""
+
+    def __init__(self, handle: int, device: torch.device):
+        self.handle = handle
+        self.device = device
+        n, ks, pairs, ptr = ctypes.c_int64(), ctypes.c_int32(), ctypes.c_int64(), ctypes.c_void_p()
+        _check(lib.spconv_map_info(handle, ctypes.byref(n), ctypes.byref(ks), ctypes.byref(pairs), ctypes.byref(ptr)))
+        self.n, self.kernel_size, self.pairs = n.value, ks.value, pairs.value
+        self._nbr_ptr = ptr.value
+
+    def neighbor_map(self) -> torch.Tensor:
+        """Copy of the dense int32 [n, 27] map (identity column for kernel size 1)."""
+        if self.kernel_size == 1:
+            return torch.arange(self.n, dtype=torch.int32, device=self.device).view(-1, 1)
+        out = torch.empty((self.n, 27), dtype=torch.int32, device=self.device)
+        if self.n:
+            # View the library-owned buffer through the CUDA array interface and copy it.
+            class _View:
+                __cuda_array_interface__ = {"shape": (self.n, 27), "typestr": "<i4",
+                                            "data": (self._nbr_ptr, False), "version": 3}
+            out.copy_(torch.as_tensor(_View(), device=self.device))
+        return out
+
+    def check(self, stream=None) -> None:
+        """Synchronise and raise if a forward kernel's bounded wait gave up."""
+        _check(lib.spconv_map_check(self.handle, _stream(stream)))
+
+    def free(self) -> None:
+        if self.handle:
+            lib.spconv_free(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass
+
+
+def spconv_build_map(coords: torch.Tensor, extent, kernel_size: int = 3, stream=None) -> SubmMap:
+    """Build the neighbour map of int32 [N, 4] (b, x, y, z) CUDA coordinates."""
+    if coords.dtype != torch.int32 or not coords.is_cuda or coords.dim() != 2 or coords.shape[1] != 4:
+        raise ValueError("coords must be a CUDA int32 tensor of shape [N, 4]")
+    coords = coords.contiguous()
+    ext = (ctypes.c_int32 * 3)(*[int(v) for v in extent])
+    handle = ctypes.c_void_p()
+    with torch.cuda.device(coords.device):
+        _check(lib.spconv_build_map(coords.data_ptr() if coords.numel() else None, coords.shape[0], ext,
+                                    kernel_size, _stream(stream), ctypes.byref(handle)))
+    return SubmMap(handle.value, coords.device)
+
+
+def spconv_subm_forward(m: SubmMap, x: torch.Tensor, w: torch.Tensor, bias: torch.Tensor | None = None,
+                        out: torch.Tensor | None = None, algo: int = ALGO_AUTO, stream=None) -> torch.Tensor:
+    """One SubMConv3d layer: x [N, Cin], w [K^3, Cin, Cout], bias [Cout] -> out [N, Cout]."""
+    if x.dtype not in _DTYPES:
+        raise ValueError("x must be float32 or bfloat16")
+    for t in (w,) + (() if bias is None else (bias,)):
+        if t.dtype != x.dtype or t.device != x.device:
+            raise ValueError("w and bias must match x in dtype and device")
+    x, w = x.contiguous(), w.contiguous()
+    bias = None if bias is None else bias.contiguous()
+    cin, cout = int(w.shape[1]), int(w.shape[2])
+    if x.shape != (m.n, cin) or w.shape[0] != m.kernel_size ** 3:
+        raise ValueError(f"shape mismatch: x {tuple(x.shape)}, w {tuple(w.shape)}, map n={m.n} k={m.kernel_size}")
+    if out is None:
+        out = torch.empty((m.n, cout), dtype=x.dtype, device=x.device)
+    elif out.shape != (m.n, cout) or out.dtype != x.dtype or not out.is_contiguous():
+        raise ValueError("out must be a contiguous [N, Cout] tensor of x's dtype")
+    if m.n == 0:
+        return out
+    with torch.cuda.device(x.device):
+        _check(lib.spconv_subm_forward_algo(m.handle, _DTYPES[x.dtype], x.data_ptr(), cin, w.data_ptr(),
+                                            None if bias is None else bias.data_ptr(), out.data_ptr(), cout,
+                                            algo, _stream(stream)))
+    return out
+
+
+def spconv_free(m: SubmMap) -> None:
+    m.free()
+
+
+def spconv_debug_set_table_slots(slots: int) -> None:
+    _check(lib.spconv_debug_set_table_slots(int(slots)))
+
+
+__all__ = ["OK", "INVALID_ARG", "UNSUPPORTED", "COORD_RANGE", "DUPLICATE", "TABLE_FULL", "OOM", "CUDA_ERROR",
+           "TIMEOUT", "SubmMap", "SpconvError", "spconv_build_map", "spconv_subm_forward", "spconv_free",
+           "spconv_debug_set_table_slots", "lib", "LIB_PATH", "EXPORTED",
+           "ALGO_AUTO", "ALGO_SIMT", "ALGO_TCGEN05"]

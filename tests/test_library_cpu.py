@@ -1,0 +1,71 @@
+"""Host-side checks of the C-ABI library that need no GPU: it loads, exports every
+symbol include/spconv.h declares, and rejects bad arguments before any device work."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "spconv.h")
+
+
+def _declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"SPCONV_API\s+[\w\s\*]+?\b(spconv_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def pkg():
+    from submanifold_sparse_convolution_submconv3d_b200 import build as b
+    b.build()
+    import submanifold_sparse_convolution_submconv3d_b200 as p
+    return p
+
+
+def test_header_declares_the_boundary():
+    syms = _declared_symbols()
+    for name in ("spconv_build_map", "spconv_subm_forward", "spconv_free"):
+        assert name in syms
+    assert len(syms) >= 8
+
+
+def test_library_exports_every_declared_symbol(pkg):
+    lib = ctypes.CDLL(pkg.LIB_PATH)
+    for name in _declared_symbols():
+        assert hasattr(lib, name), name
+    assert set(_declared_symbols()) == set(pkg.EXPORTED)
+    out = subprocess.run(["nm", "-D", "--defined-only", pkg.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (spconv_\w+)", out))
+    assert exported == set(_declared_symbols())
+
+
+def test_host_validation_without_device_work(pkg):
+    lib = pkg.lib
+    handle = ctypes.c_void_p()
+    ext = (ctypes.c_int32 * 3)(4, 4, 4)
+    assert lib.spconv_build_map(None, 0, ext, 5, None, ctypes.byref(handle)) == pkg.INVALID_ARG
+    assert b"kernel_size" in lib.spconv_last_error()
+    bad_ext = (ctypes.c_int32 * 3)(0, 4, 4)
+    assert lib.spconv_build_map(None, 0, bad_ext, 3, None, ctypes.byref(handle)) == pkg.INVALID_ARG
+    big_ext = (ctypes.c_int32 * 3)(70000, 4, 4)
+    assert lib.spconv_build_map(None, 0, big_ext, 3, None, ctypes.byref(handle)) == pkg.INVALID_ARG
+    assert lib.spconv_build_map(None, -1, ext, 3, None, ctypes.byref(handle)) == pkg.INVALID_ARG
+    assert lib.spconv_build_map(None, 5, ext, 3, None, ctypes.byref(handle)) == pkg.INVALID_ARG  # null coords
+    assert lib.spconv_build_map(None, 1 << 31, ext, 3, None, ctypes.byref(handle)) == pkg.INVALID_ARG
+    assert lib.spconv_build_map(None, 0, ext, 3, None, None) == pkg.INVALID_ARG
+    assert handle.value is None
+    assert lib.spconv_map_info(None, None, None, None, None) == pkg.INVALID_ARG
+    assert lib.spconv_free(None) == pkg.OK
+    assert lib.spconv_subm_forward(None, 1, None, 16, None, None, None, 16, None) == pkg.INVALID_ARG
+    assert lib.spconv_debug_set_table_slots(3) == pkg.INVALID_ARG
+    assert lib.spconv_debug_set_table_slots(0) == pkg.OK
+
+
+def test_python_binding_rejects_bad_tensors(pkg):
+    import torch
+    with pytest.raises(ValueError):
+        pkg.spconv_build_map(torch.zeros((3, 4), dtype=torch.int64), (4, 4, 4))
+    with pytest.raises(ValueError):
+        pkg.spconv_build_map(torch.zeros((3, 3), dtype=torch.int32), (4, 4, 4))
