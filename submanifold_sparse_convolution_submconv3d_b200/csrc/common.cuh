@@ -5,7 +5,7 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
-#include "../../include/spconv.h"
+#include "spconv.h"
 
 namespace spconv {
 

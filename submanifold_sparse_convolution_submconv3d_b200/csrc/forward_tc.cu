@@ -10,7 +10,7 @@
 // One CTA owns kTileRows consecutive output rows and one block of 64 or 128
 // output channels.  Tensor memory (TMEM, 128 lanes x 512 fp32 columns) holds
 //   * the accumulator: lane = output channel, column = output row of the tile;
-//   * two scratch buffers of kScratchCols columns.
+//   * two scratch buffers of kScratchCols columns and a few dummy columns.
 // The centre offset (every row is its own neighbour) is one dense MMA per 128
 // rows straight into the accumulator.  For every other offset the rows of the
 // tile that have a neighbour there are compacted into a list; their neighbour
@@ -20,11 +20,15 @@
 // (tcgen05.ld / tcgen05.st, no atomics).  Weights W_k arrive by TMA.  At the
 // end each output row is written exactly once, with bias, rounded to bf16.
 //
-// Warp roles (320 threads):
+// Warp roles (576 threads):
 //   warp 0      TMA producer of weight tiles (A operand)
 //   warp 1      TMEM allocator and tcgen05.mma issuer
 //   warps 2-5   gather producers of feature rows (B operand)
-//   warps 6-9   scratch -> accumulator fold, then the epilogue
+//   warps 6-17  scratch -> accumulator fold, then the epilogue: three warps per
+//               TMEM lane quarter, each owning the tile rows of one residue mod 3,
+//               so no accumulator column is touched by two warps of a quarter.
+//               Narrow TMEM accesses are issued without per-element branches;
+//               padding entries go to dedicated dummy columns.
 // Every spin-wait is bounded: after kWaitTimeoutNs the kernel records
 // kFwdErrTimeout in the map's error word, stops issuing work, lets copies in
 // flight land, frees its TMEM and returns.
@@ -39,13 +43,18 @@ namespace {
 using namespace sm100;
 
 constexpr int kTileRows = 384;
-constexpr int kScratchCols = 64;
+constexpr int kClasses = 3;                       // rows split by r % 3 between fold warps
+constexpr int kClassRows = kTileRows / kClasses;  // 128
+constexpr int kScratchCols = 48;
 constexpr int kCentreCols = 128;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kScratchCol0 = kTileRows;  // scratch buffer b at column 384 + 64 b
-constexpr int kThreads = 320;
+constexpr uint32_t kScratchCol0 = kTileRows;      // scratch buffer b at column 384 + 48 b
+constexpr uint32_t kDummyCol0 = kScratchCol0 + 2 * kScratchCols;  // 480..495: fold padding targets
 constexpr int kWarpTma = 0, kWarpMma = 1, kWarpGather0 = 2, kWarpFold0 = 6;
-constexpr int kGatherThreads = 128;
+constexpr int kGatherWarps = 4, kFoldWarps = 12;
+constexpr int kThreads = 32 * (kWarpFold0 + kFoldWarps);  // 576
+constexpr int kGatherThreads = 32 * kGatherWarps;
+constexpr int kFoldGroup = 16;
 constexpr uint64_t kWaitTimeoutNs = 4000000000ull;
 constexpr int kMaxSmem = 232448;  // 227 KB opt-in limit per CTA on sm_100
 
@@ -59,7 +68,7 @@ struct Layout {
     static constexpr int kRowsPerPass = kGatherThreads / kThreadsPerRow;
     static constexpr int kABytes = BM * KC * 2;                   // weight tile per stage
     static constexpr int kAPad = round_up(kABytes, 1024);
-    static constexpr int kBPad = round_up(128 * kRowBytes, 1024); // up to 128 gathered rows
+    static constexpr int kBPad = round_up(kCentreCols * kRowBytes, 1024);  // up to 128 gathered rows
     static constexpr int kStageBytes = kAPad + kBPad;
     static constexpr uint32_t kSwizzleMask = kRowBytes / 16 - 1;
     static constexpr uint32_t kBLayout = KC == 64 ? 2u : (KC == 32 ? 4u : 6u);  // 128/64/32-byte swizzle
@@ -68,9 +77,10 @@ struct Layout {
     static constexpr int kChPerWarp = BM / 4;                     // channels of one TMEM lane quarter
 
     static constexpr int kNbrBytes = kTileRows * kVol3 * 4;
-    static constexpr int kListBytes = kVol3 * kTileRows * 2;
-    static constexpr int kOutStageBytes = 4 * 32 * kChPerWarp * 2;
-    static constexpr int kMetaBytes = kNbrBytes + kListBytes + 128 + kOutStageBytes + 64 * 8 + 16;
+    static constexpr int kListBytes = kVol3 * kClasses * kClassRows * 2;
+    static constexpr int kCntBytes = round_up(kVol3 * kClasses * 4, 16);
+    static constexpr int kOutStageBytes = kFoldWarps * 32 * kChPerWarp * 2;
+    static constexpr int kMetaBytes = kNbrBytes + kListBytes + kCntBytes + kOutStageBytes + 64 * 8 + 16;
 
     static int stages() {
         int s = (kMaxSmem - 1024 - kMetaBytes) / kStageBytes;
@@ -92,15 +102,27 @@ struct Params {
     int stages;
 };
 
-// A unit of MMA work: one offset, up to 128 (centre) or 64 (other) columns.
+// A unit of MMA work: one offset, up to 128 (centre) or 48 (other) columns.
 struct Job {
-    int k;       // offset index into the tile metadata (13 = centre for kernel size 3)
-    int kw;      // weight slice index (k for kernel size 3, 0 for kernel size 1)
-    int first;   // first row (centre) or first list entry (other offsets)
+    int k;       // offset (13 = centre for kernel size 3; 0 for kernel size 1)
+    int first;   // first row (centre) or first entry of the offset's list (other offsets)
     int n;       // valid columns
     int ncols;   // MMA N (n rounded up)
     bool centre;
 };
+
+// Per-offset hit lists.  Offset k's list is the concatenation of three classes
+// (rows r with r % 3 == 0, 1, 2), each sorted by row; class c of offset k is
+// lists[(3k + c) * 128 + i], i < cnt[3k + c].
+__device__ __forceinline__ int list_total(const int* cnt, int k) {
+    return cnt[3 * k] + cnt[3 * k + 1] + cnt[3 * k + 2];
+}
+__device__ __forceinline__ int list_row(const uint16_t* lists, const int* cnt, int k, int e) {
+    const int c0 = cnt[3 * k], c1 = cnt[3 * k + 1];
+    const int c = (e >= c0) + (e >= c0 + c1);
+    const int idx = e - (c >= 1 ? c0 : 0) - (c >= 2 ? c1 : 0);
+    return lists[(3 * k + c) * kClassRows + idx];
+}
 
 // Enumerates the jobs of a tile in issue order: centre slices, then offsets 0..26
 // (skipping the centre) split into kScratchCols-wide parts.  Every role walks the
@@ -108,7 +130,7 @@ struct Job {
 struct JobIter {
     const int* cnt;
     int t_eff, kvol, nalign;
-    int k, first;  // position
+    int k, first, total;
     __device__ void start() {
         k = -1;
         first = 0;
@@ -117,7 +139,6 @@ struct JobIter {
         if (k == -1) {
             if (first < t_eff) {
                 j.k = kvol == kVol3 ? kCentre : 0;
-                j.kw = j.k;
                 j.first = first;
                 j.n = min(kCentreCols, t_eff - first);
                 j.ncols = round_up(j.n, nalign);
@@ -128,13 +149,13 @@ struct JobIter {
             if (kvol != kVol3) return false;
             k = 0;
             first = 0;
+            total = list_total(cnt, 0);
         }
         while (k < kVol3) {
-            if (k != kCentre && first < cnt[k]) {
+            if (k != kCentre && first < total) {
                 j.k = k;
-                j.kw = k;
                 j.first = first;
-                j.n = min(kScratchCols, cnt[k] - first);
+                j.n = min(kScratchCols, total - first);
                 j.ncols = round_up(j.n, nalign);
                 j.centre = false;
                 first += kScratchCols;
@@ -142,6 +163,7 @@ struct JobIter {
             }
             ++k;
             first = 0;
+            if (k < kVol3) total = list_total(cnt, k);
         }
         return false;
     }
@@ -172,6 +194,10 @@ __device__ __forceinline__ bool warp_wait_bar(uint32_t bar, uint32_t parity, vol
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
+__device__ __forceinline__ void named_barrier(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 template <int BM, int KC>
 __global__ void __launch_bounds__(kThreads, 1)
     k_subm_tc(const __grid_constant__ CUtensorMap wmap, const Params p) {
@@ -183,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int32_t* nbr_s = reinterpret_cast<int32_t*>(smem + S * L::kStageBytes);
     uint16_t* lists = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(nbr_s) + L::kNbrBytes);
     int* cnt = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(lists) + L::kListBytes);
-    __nv_bfloat16* out_stage = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(cnt) + 128);
+    __nv_bfloat16* out_stage = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(cnt) + L::kCntBytes);
     uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(out_stage) + L::kOutStageBytes);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 6);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -198,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int cblk = blockIdx.y;
     const int nchunks = p.cin / KC;
 
-    // ---- set-up: barriers, TMEM, neighbour rows of the tile
+    // ---- set-up: barriers, TMEM, neighbour rows of the tile (cp.async, 16 B)
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(full0 + 8 * s, 1 + kGatherThreads);
@@ -206,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(sfull0 + 8 * b, 1);
-            mbar_init(sempty0 + 8 * b, 4);
+            mbar_init(sempty0 + 8 * b, kFoldWarps);
         }
         mbar_init(accfull, 1);
         mbar_init(drain, 1);
@@ -219,33 +245,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_relinquish();
     }
     if (p.kvol == kVol3) {
-        const int total = kTileRows * kVol3, valid = t_eff * kVol3;
+        // rows row0 .. row0 + t_eff of the map are contiguous: t_eff * 108 bytes,
+        // 16-byte aligned because kTileRows * 108 is a multiple of 16.
+        const int words = t_eff * kVol3;
+        const int vecs = words / 4;
         const int32_t* src = p.nbr + row0 * kVol3;
-        for (int i = threadIdx.x; i < total; i += kThreads) nbr_s[i] = i < valid ? __ldg(src + i) : -1;
+        const uint32_t dst = smem_addr(nbr_s);
+        for (int i = threadIdx.x; i < vecs; i += kThreads) cp_async_16(dst + 16 * i, src + 4 * i, 16);
+        for (int i = 4 * vecs + threadIdx.x; i < words; i += kThreads) nbr_s[i] = __ldg(src + i);
+        cp_async_wait_all();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    // ---- per-offset lists of tile rows that have a neighbour (sorted by row)
+    // ---- per-offset, per-class lists of tile rows that have a neighbour
     if (p.kvol == kVol3 && warp >= kWarpGather0) {
-        for (int k = warp - kWarpGather0; k < kVol3; k += kThreads / 32 - kWarpGather0) {
-            if (k == kCentre) continue;
-            int c = 0;
-            for (int base = 0; base < t_eff; base += 32) {
-                const int r = base + lane;
+        constexpr int kListWarps = kThreads / 32 - kWarpGather0;
+        for (int u = warp - kWarpGather0; u < (kVol3 - 1) * kClasses; u += kListWarps) {
+            const int ks = u / kClasses, c = u - ks * kClasses;
+            const int k = ks < kCentre ? ks : ks + 1;
+            int n = 0;
+            for (int base = 0; base < kClassRows; base += 32) {
+                const int r = c + kClasses * (base + lane);
                 const bool hit = r < t_eff && nbr_s[r * kVol3 + k] >= 0;
                 const unsigned b = __ballot_sync(0xffffffffu, hit);
-                if (hit) lists[k * kTileRows + c + __popc(b & ((1u << lane) - 1u))] = (uint16_t)r;
-                c += __popc(b);
+                if (hit) lists[(3 * k + c) * kClassRows + n + __popc(b & ((1u << lane) - 1u))] = (uint16_t)r;
+                n += __popc(b);
             }
-            if (lane == 0) cnt[k] = c;
+            if (lane == 0) cnt[3 * k + c] = n;
         }
     }
     __syncthreads();
 
-    JobIter it_jobs{cnt, t_eff, p.kvol, L::kNAlign, 0, 0};
+    JobIter it_jobs{cnt, t_eff, p.kvol, L::kNAlign, 0, 0, 0};
     Job job;
     bool aborted = false;
 
@@ -264,7 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     const uint32_t a_dst = smem_addr(stages + s * L::kStageBytes);
                     mbar_arrive_expect_tx(full0 + 8 * s, L::kABytes);
-                    const int y = job.kw * p.cin + c * KC;
+                    const int y = job.k * p.cin + c * KC;
                     for (int box = 0; box < BM / 64; ++box)
                         tma_load_2d(a_dst + box * KC * 128, &wmap, cblk * BM + box * 64, y, full0 + 8 * s);
                 }
@@ -277,7 +311,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             int it = 0, sj = 0;
             it_jobs.start();
             while (!aborted && it_jobs.next(job)) {
-                uint32_t d = tmem + (job.centre ? (uint32_t)job.first : kScratchCol0 + (uint32_t)(sj & 1) * kScratchCols);
+                const uint32_t d =
+                    tmem + (job.centre ? (uint32_t)job.first : kScratchCol0 + (uint32_t)(sj & 1) * kScratchCols);
                 if (!job.centre) {
                     if (!wait_bar(sempty0 + 8 * (sj & 1), ((uint32_t)(sj >> 1) & 1u) ^ 1u, abort_flag, p.err)) {
                         aborted = true;
@@ -328,7 +363,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         int it = 0;
         it_jobs.start();
         while (!aborted && it_jobs.next(job)) {
-            const uint16_t* list = lists + job.k * kTileRows + job.first;
             for (int c = 0; c < nchunks; ++c, ++it) {
                 const int s = it % S;
                 const uint32_t ph = (uint32_t)(it / S) & 1u;
@@ -346,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (job.centre) {
                             j = row0 + job.first + pr;
                         } else {
-                            const int r = list[pr];
+                            const int r = list_row(lists, cnt, job.k, job.first + pr);
                             j = nbr_s[r * kVol3 + job.k];
                         }
                         src = p.x + j * p.cin + col_off;
@@ -361,7 +395,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         cp_async_wait_all();
     } else {
         // ------------------------------------------------ fold scratch -> accumulator, then epilogue
-        const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
+        // Warp (quarter, sub) owns TMEM lanes [32*quarter, +32) and the tile rows
+        // r with r % 3 == sub, so every accumulator column is only ever touched by
+        // one warp per lane quarter.
+        const int quarter = warp & 3;
+        const int sub = (warp - kWarpFold0) >> 2;
         const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
         int sj = 0;
         it_jobs.start();
@@ -374,40 +412,53 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after();
             const uint32_t scr = tmem + lane_base + kScratchCol0 + (uint32_t)b * kScratchCols;
-            const uint16_t* list = lists + job.k * kTileRows + job.first;
-            for (int p0 = 0; p0 < job.n; p0 += 8) {
-                float v[8], a[8];
-                uint32_t col[8];
-                tmem_ld_x8(scr + p0, v);
+            const int k = job.k;
+            const int cls_start = (sub >= 1 ? cnt[3 * k] : 0) + (sub >= 2 ? cnt[3 * k + 1] : 0);
+            const int lo = max(job.first, cls_start);
+            const int hi = min(job.first + job.n, cls_start + cnt[3 * k + sub]);
+            const uint16_t* lst = lists + (3 * k + sub) * kClassRows;
+            bool released = false;
+            for (int g0 = lo; g0 < hi; g0 += kFoldGroup) {
+                float v[kFoldGroup], a[kFoldGroup];
+                uint32_t col[kFoldGroup];
+                tmem_ld_x16(scr + (uint32_t)(g0 - job.first), v);
+                if (g0 == lo) tmem_wait_st();  // this warp's stores of the previous job have landed
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    if (p0 + i < job.n) {
-                        col[i] = tmem + lane_base + list[p0 + i];
-                        tmem_ld_x1(col[i], a[i]);
-                    }
+                for (int i = 0; i < kFoldGroup; ++i) {
+                    const int e = g0 + i;
+                    const uint32_t r = lst[min(e, hi - 1) - cls_start];
+                    col[i] = tmem + lane_base + (e < hi ? r : kDummyCol0 + (uint32_t)i);
+                    tmem_ld_x1(col[i], a[i]);
                 }
                 tmem_wait_ld();
+                if (g0 + kFoldGroup >= hi) {  // last group: the scratch buffer has been read
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(sempty0 + 8 * b);
+                    released = true;
+                }
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    if (p0 + i < job.n) tmem_st_x1(col[i], a[i] + v[i]);
+                for (int i = 0; i < kFoldGroup; ++i) tmem_st_x1(col[i], a[i] + v[i]);
             }
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(sempty0 + 8 * b);
+            if (!released) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(sempty0 + 8 * b);
+            }
             ++sj;
         }
+        tmem_wait_st();
+        tc_fence_before();
+        named_barrier(1, 32 * kFoldWarps);  // every fold store has landed before any epilogue read
         if (!aborted && warp_wait_bar(accfull, 0, abort_flag, p.err)) {
             tc_fence_after();
-            // channel held by this thread's TMEM lane
             const bool lane_ok = lane < L::kChPerWarp;
-            const int ch_local = quarter * L::kChPerWarp + lane;  // channel within the block
-            const int ch = cblk * BM + ch_local;
+            const int ch_base = cblk * BM + quarter * L::kChPerWarp;
+            const int ch = ch_base + lane;
             const float bv = (p.bias && lane_ok && ch < p.cout) ? __bfloat162float(p.bias[ch]) : 0.0f;
             __nv_bfloat16* stg = out_stage + (warp - kWarpFold0) * 32 * L::kChPerWarp;
             constexpr int kVecPerRow = L::kChPerWarp * 2 / 16;
-            const int ch_base = cblk * BM + quarter * L::kChPerWarp;
-            for (int col = 0; col < t_eff; col += 32) {
+            for (int col = 32 * sub; col < t_eff; col += 32 * kClasses) {
                 float v[32];
                 tmem_ld_x32(tmem + lane_base + (uint32_t)col, v);
                 tmem_wait_ld();

@@ -183,17 +183,20 @@ def test_uniform_ten_layers_chained_sampled(sp):
         m.free()
 
 
-def test_uniform_full_output_simt_vs_tcgen05(sp):
-    """Every row of one full-size layer: tensor-core kernel vs the CUDA-core kernel."""
+def test_uniform_full_output_every_row(sp):
+    """Every row of one full-size layer of the pages' shape, both kernels, against
+    the fp64 oracle over the whole output."""
     wl = workloads.make_workload("uniform", 0, n_layers=1)
+    layer = wl.layers[0]
     m = sp.spconv_build_map(coords_dev(wl.coords), wl.grid, 3)
     try:
-        x, w, b = to_dev(wl.x, "bf16"), to_dev(wl.layers[0].w, "bf16"), to_dev(wl.layers[0].bias, "bf16")
-        tc = sp.spconv_subm_forward(m, x, w, b, algo=sp.ALGO_TCGEN05).float()
-        simt = sp.spconv_subm_forward(m, x, w, b, algo=sp.ALGO_SIMT).float()
+        x, w, b = to_dev(wl.x, "bf16"), to_dev(layer.w, "bf16"), to_dev(layer.bias, "bf16")
+        tc = sp.spconv_subm_forward(m, x, w, b, algo=sp.ALGO_TCGEN05)
+        simt = sp.spconv_subm_forward(m, x, w, b, algo=sp.ALGO_SIMT)
         m.check()
-        rms = float(simt.pow(2).mean().sqrt())
-        assert float((tc - simt).abs().max()) / rms <= 2e-2
+        ref = oracle.forward(m.neighbor_map().cpu().numpy(), wl.x, layer.w, layer.bias)
+        assert_close(tc, ref, "bf16")
+        assert_close(simt, ref, "bf16")
     finally:
         m.free()
 
