@@ -31,6 +31,20 @@ struct BuildFlags {
 constexpr int kVol3 = 27;
 constexpr int kCentre = 13;
 
+// Tile metadata (built with the map, kernel size 3): the rows are cut into tiles
+// of kTileRows consecutive rows; for every tile and every non-centre offset the
+// tile rows with an active neighbour there are listed, split into three classes
+// by row % 3 and sorted by row within a class.  "Units" are (offset, class)
+// pairs in offset-major order, offsets 0..26 without the centre: unit
+// u = 3 * ks + c with ks = k < 13 ? k : k - 1.
+constexpr int kTileRows = 384;
+constexpr int kTileClasses = 3;
+constexpr int kTileUnits = (kVol3 - 1) * kTileClasses;  // 78
+constexpr int kTileCountStride = 80;                    // int32 counts per tile (78 used), 320 bytes
+constexpr int kTileEntryAlign = 8;                      // each tile's entries start on a multiple of 8
+
+__host__ __device__ inline int64_t num_tiles(int64_t n) { return (n + kTileRows - 1) / kTileRows; }
+
 // The map handle (defined here so the launchers can read it).
 struct MapData {
     int64_t n = 0;
@@ -38,6 +52,13 @@ struct MapData {
     int32_t extent[3] = {0, 0, 0};
     int64_t pairs = 0;
     int32_t* nbr = nullptr;        // device [n, 27] (kernel size 3), else null
+    // tile metadata (kernel size 3): counts [ntiles][kTileCountStride], entry offsets
+    // [ntiles + 1] (multiples of kTileEntryAlign), local rows and neighbour rows per entry
+    int32_t* tile_counts = nullptr;
+    int64_t* tile_off = nullptr;
+    uint16_t* pair_r = nullptr;
+    int32_t* pair_j = nullptr;
+    int64_t tile_entries = 0;
     unsigned int* fwd_err = nullptr;  // device word: forward-kernel error bits
     int device = 0;
     int num_sms = 0;
@@ -47,6 +68,13 @@ struct MapData {
 cudaError_t launch_build_map(const int32_t* coords, int64_t n, const int32_t extent[3], int32_t kernel_size,
                              unsigned long long* table, uint64_t slots, int32_t* nbr, BuildFlags* flags,
                              cudaStream_t stream);
+
+// Tile metadata in two passes: counts + offsets (then the caller reads the total
+// and allocates the entry arrays), then the entries.
+cudaError_t launch_tile_count(const int32_t* nbr, int64_t n, int32_t* tile_counts, int64_t* tile_off,
+                              cudaStream_t stream);
+cudaError_t launch_tile_fill(const int32_t* nbr, int64_t n, const int32_t* tile_counts, const int64_t* tile_off,
+                             uint16_t* pair_r, int32_t* pair_j, cudaStream_t stream);
 
 cudaError_t launch_forward_simt(const MapData& m, spconv_dtype_t dtype, const void* x, int cin, const void* w,
                                 const void* bias, void* out, int cout, cudaStream_t stream);

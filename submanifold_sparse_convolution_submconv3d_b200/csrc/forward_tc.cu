@@ -14,8 +14,8 @@
 // The centre offset (every row is its own neighbour) is one dense MMA per 128
 // rows straight into the accumulator.  For every other offset the rows of the
 // tile that have a neighbour there are compacted into a list; their neighbour
-// feature rows are gathered (cp.async, 16 B, zero-filled padding) into a
-// swizzled shared-memory tile and multiplied into a scratch buffer, and four
+// feature rows are gathered (cp.async, 16 B, zero-filled holes and padding)
+// into a swizzled shared-memory tile and multiplied into a scratch buffer, and fold
 // warps then add each scratch column into the accumulator column of its row
 // (tcgen05.ld / tcgen05.st, no atomics).  Weights W_k arrive by TMA.  At the
 // end each output row is written exactly once, with bias, rounded to bf16.
@@ -42,9 +42,8 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kTileRows = 384;
-constexpr int kClasses = 3;                       // rows split by r % 3 between fold warps
-constexpr int kClassRows = kTileRows / kClasses;  // 128
+constexpr int kClasses = kTileClasses;           // rows split by r % 3 between fold warps
+constexpr int kMaxEntries = (kVol3 - 1) * kTileRows;  // tile metadata entries, worst case
 constexpr int kScratchCols = 48;
 constexpr int kCentreCols = 128;
 constexpr uint32_t kTmemCols = 512;
@@ -66,21 +65,21 @@ struct Layout {
     static constexpr int kRowBytes = KC * 2;                      // one gathered row chunk
     static constexpr int kThreadsPerRow = kRowBytes / 16;
     static constexpr int kRowsPerPass = kGatherThreads / kThreadsPerRow;
+    static constexpr uint32_t kSwizzleMask = kRowBytes / 16 - 1;
     static constexpr int kABytes = BM * KC * 2;                   // weight tile per stage
     static constexpr int kAPad = round_up(kABytes, 1024);
     static constexpr int kBPad = round_up(kCentreCols * kRowBytes, 1024);  // up to 128 gathered rows
     static constexpr int kStageBytes = kAPad + kBPad;
-    static constexpr uint32_t kSwizzleMask = kRowBytes / 16 - 1;
     static constexpr uint32_t kBLayout = KC == 64 ? 2u : (KC == 32 ? 4u : 6u);  // 128/64/32-byte swizzle
     static constexpr uint32_t kBSbo = 8 * kRowBytes;
     static constexpr int kNAlign = BM == 128 ? 16 : 8;
     static constexpr int kChPerWarp = BM / 4;                     // channels of one TMEM lane quarter
 
-    static constexpr int kNbrBytes = kTileRows * kVol3 * 4;
-    static constexpr int kListBytes = kVol3 * kClasses * kClassRows * 2;
-    static constexpr int kCntBytes = round_up(kVol3 * kClasses * 4, 16);
+    static constexpr int kEntryJBytes = kMaxEntries * 4;           // neighbour rows of the tile's entries
+    static constexpr int kEntryRBytes = kMaxEntries * 2;           // local rows of the tile's entries
+    static constexpr int kCntBytes = 2 * kTileCountStride * 4;     // unit counts, then unit starts
     static constexpr int kOutStageBytes = kFoldWarps * 32 * kChPerWarp * 2;
-    static constexpr int kMetaBytes = kNbrBytes + kListBytes + kCntBytes + kOutStageBytes + 64 * 8 + 16;
+    static constexpr int kMetaBytes = kEntryJBytes + kEntryRBytes + kCntBytes + kOutStageBytes + 64 * 8 + 32;
 
     static int stages() {
         int s = (kMaxSmem - 1024 - kMetaBytes) / kStageBytes;
@@ -90,7 +89,10 @@ struct Layout {
 };
 
 struct Params {
-    const int32_t* nbr;  // [n, 27] or null for kernel size 1
+    const int32_t* tile_counts;  // tile metadata (null for kernel size 1)
+    const int64_t* tile_off;
+    const uint16_t* pair_r;
+    const int32_t* pair_j;
     int64_t n;
     int kvol;
     const __nv_bfloat16* x;
@@ -105,40 +107,42 @@ struct Params {
 // A unit of MMA work: one offset, up to 128 (centre) or 48 (other) columns.
 struct Job {
     int k;       // offset (13 = centre for kernel size 3; 0 for kernel size 1)
+    int ks;      // index among the 26 non-centre offsets (other offsets)
+    int base;    // flat index of the offset's first entry in the tile metadata
     int first;   // first row (centre) or first entry of the offset's list (other offsets)
     int n;       // valid columns
     int ncols;   // MMA N (n rounded up)
     bool centre;
 };
 
-// Per-offset hit lists.  Offset k's list is the concatenation of three classes
-// (rows r with r % 3 == 0, 1, 2), each sorted by row; class c of offset k is
-// lists[(3k + c) * 128 + i], i < cnt[3k + c].
-__device__ __forceinline__ int list_total(const int* cnt, int k) {
-    return cnt[3 * k] + cnt[3 * k + 1] + cnt[3 * k + 2];
-}
-__device__ __forceinline__ int list_row(const uint16_t* lists, const int* cnt, int k, int e) {
-    const int c0 = cnt[3 * k], c1 = cnt[3 * k + 1];
-    const int c = (e >= c0) + (e >= c0 + c1);
-    const int idx = e - (c >= 1 ? c0 : 0) - (c >= 2 ? c1 : 0);
-    return lists[(3 * k + c) * kClassRows + idx];
-}
-
-// Enumerates the jobs of a tile in issue order: centre slices, then offsets 0..26
-// (skipping the centre) split into kScratchCols-wide parts.  Every role walks the
-// same sequence.
+// Per-offset hit lists come from the tile metadata built with the map: offset
+// k's entries are the concatenation of its three classes (rows r with r % 3 ==
+// 0, 1, 2, each sorted by row), flat indices ustart[3 ks] .. ustart[3 ks + 3).
+// Enumerates the jobs of a tile in issue order: centre slices, then the other 26
+// offsets, each split into kScratchCols-wide parts.  The order of the 26 offsets
+// is rotated per CTA (`rot`) so that CTAs running at the same time request
+// different weight tiles instead of all reading the same L2 lines.  Every role
+// of a CTA walks the same sequence.
 struct JobIter {
-    const int* cnt;
-    int t_eff, kvol, nalign;
-    int k, first, total;
+    const int* ustart;  // unit starts, ustart[kTileUnits] = number of entries
+    int t_eff, kvol, nalign, rot;
+    int ki, k, ks, first, total;  // ki: position among the 26 non-centre offsets
     __device__ void start() {
-        k = -1;
+        ki = -1;
+        first = 0;
+    }
+    __device__ void set_offset() {
+        ks = (ki + rot) % (kVol3 - 1);
+        k = ks < kCentre ? ks : ks + 1;
+        total = ustart[3 * ks + 3] - ustart[3 * ks];
         first = 0;
     }
     __device__ bool next(Job& j) {
-        if (k == -1) {
+        if (ki == -1) {
             if (first < t_eff) {
                 j.k = kvol == kVol3 ? kCentre : 0;
+                j.ks = 0;
+                j.base = 0;
                 j.first = first;
                 j.n = min(kCentreCols, t_eff - first);
                 j.ncols = round_up(j.n, nalign);
@@ -147,13 +151,14 @@ struct JobIter {
                 return true;
             }
             if (kvol != kVol3) return false;
-            k = 0;
-            first = 0;
-            total = list_total(cnt, 0);
+            ki = 0;
+            set_offset();
         }
-        while (k < kVol3) {
-            if (k != kCentre && first < total) {
+        while (ki < kVol3 - 1) {
+            if (first < total) {
                 j.k = k;
+                j.ks = ks;
+                j.base = ustart[3 * ks];
                 j.first = first;
                 j.n = min(kScratchCols, total - first);
                 j.ncols = round_up(j.n, nalign);
@@ -161,19 +166,21 @@ struct JobIter {
                 first += kScratchCols;
                 return true;
             }
-            ++k;
-            first = 0;
-            if (k < kVol3) total = list_total(cnt, k);
+            if (++ki < kVol3 - 1) set_offset();
         }
         return false;
     }
 };
 
+// Bounded wait on an mbarrier phase.  `backoff` lets a non-critical waiter sleep
+// between polls so that it does not take issue slots from the MMA issuer.
+template <bool backoff = false>
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                          unsigned int* err) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 1;; ++i) {
+        if (backoff) __nanosleep(64);
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 63) == 0) {
             if (*abort_flag) return false;
@@ -186,17 +193,26 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
     }
 }
 
-// Whole-warp wait: lane 0 polls, the result is broadcast.
-__device__ __forceinline__ bool warp_wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                              unsigned int* err) {
-    int ok = 0;
-    if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, abort_flag, err) ? 1 : 0;
-    return __shfl_sync(0xffffffffu, ok, 0) != 0;
-}
-
 __device__ __forceinline__ void named_barrier(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
+
+// Group wait: one thread of the group polls the mbarrier, the whole group then
+// meets at a hardware named barrier (blocked warps take no issue slots).  The
+// result travels through one of two alternating shared-memory slots.
+struct GroupWait {
+    int barrier_id, nthreads;
+    bool leader;
+    volatile int* slots;  // two ints
+    int phase;
+    __device__ bool operator()(uint32_t bar, uint32_t parity, volatile int* abort_flag, unsigned int* err) {
+        volatile int* slot = slots + (phase & 1);
+        ++phase;
+        if (leader) *slot = wait_bar<true>(bar, parity, abort_flag, err) ? 1 : 0;
+        named_barrier(barrier_id, nthreads);
+        return *slot != 0;
+    }
+};
 
 template <int BM, int KC>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -206,13 +222,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int S = p.stages;
     uint8_t* stages = smem;
-    int32_t* nbr_s = reinterpret_cast<int32_t*>(smem + S * L::kStageBytes);
-    uint16_t* lists = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(nbr_s) + L::kNbrBytes);
-    int* cnt = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(lists) + L::kListBytes);
+    int32_t* pj_s = reinterpret_cast<int32_t*>(smem + S * L::kStageBytes);
+    uint16_t* pr_s = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(pj_s) + L::kEntryJBytes);
+    int* cnt = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(pr_s) + L::kEntryRBytes);
+    int* ustart = cnt + kTileCountStride;
     __nv_bfloat16* out_stage = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(cnt) + L::kCntBytes);
     uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(out_stage) + L::kOutStageBytes);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 6);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* wait_slots = abort_flag + 1;  // 2 for the gather group, 2 for the fold group
 
     const uint32_t full0 = smem_addr(bars), empty0 = smem_addr(bars + S);
     const uint32_t sfull0 = smem_addr(bars + 2 * S), sempty0 = smem_addr(bars + 2 * S + 2);
@@ -245,14 +263,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_relinquish();
     }
     if (p.kvol == kVol3) {
-        // rows row0 .. row0 + t_eff of the map are contiguous: t_eff * 108 bytes,
-        // 16-byte aligned because kTileRows * 108 is a multiple of 16.
-        const int words = t_eff * kVol3;
-        const int vecs = words / 4;
-        const int32_t* src = p.nbr + row0 * kVol3;
-        const uint32_t dst = smem_addr(nbr_s);
-        for (int i = threadIdx.x; i < vecs; i += kThreads) cp_async_16(dst + 16 * i, src + 4 * i, 16);
-        for (int i = 4 * vecs + threadIdx.x; i < words; i += kThreads) nbr_s[i] = __ldg(src + i);
+        // The tile's metadata: unit counts (320 B) and entries (local row, neighbour
+        // row); every tile's entries start on a multiple of 8, so all copies are
+        // 16-byte aligned.
+        const int64_t e0 = p.tile_off[blockIdx.x], ne = p.tile_off[blockIdx.x + 1] - e0;
+        const uint32_t cnt_dst = smem_addr(cnt), pj_dst = smem_addr(pj_s), pr_dst = smem_addr(pr_s);
+        const int32_t* cnt_src = p.tile_counts + (int64_t)blockIdx.x * kTileCountStride;
+        for (int i = threadIdx.x; i < kTileCountStride / 4; i += kThreads) cp_async_16(cnt_dst + 16 * i, cnt_src + 4 * i, 16);
+        for (int i = threadIdx.x; i < ne / 4; i += kThreads) cp_async_16(pj_dst + 16 * i, p.pair_j + e0 + 4 * i, 16);
+        for (int i = threadIdx.x; i < ne / 8; i += kThreads) cp_async_16(pr_dst + 16 * i, p.pair_r + e0 + 8 * i, 16);
         cp_async_wait_all();
     }
     tc_fence_before();
@@ -260,26 +279,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    // ---- per-offset, per-class lists of tile rows that have a neighbour
-    if (p.kvol == kVol3 && warp >= kWarpGather0) {
-        constexpr int kListWarps = kThreads / 32 - kWarpGather0;
-        for (int u = warp - kWarpGather0; u < (kVol3 - 1) * kClasses; u += kListWarps) {
-            const int ks = u / kClasses, c = u - ks * kClasses;
-            const int k = ks < kCentre ? ks : ks + 1;
-            int n = 0;
-            for (int base = 0; base < kClassRows; base += 32) {
-                const int r = c + kClasses * (base + lane);
-                const bool hit = r < t_eff && nbr_s[r * kVol3 + k] >= 0;
-                const unsigned b = __ballot_sync(0xffffffffu, hit);
-                if (hit) lists[(3 * k + c) * kClassRows + n + __popc(b & ((1u << lane) - 1u))] = (uint16_t)r;
-                n += __popc(b);
+    // ---- flat start of every (offset, class) unit
+    if (p.kvol == kVol3 && warp == 0) {
+        int run = 0;
+        for (int base = 0; base < kTileUnits; base += 32) {
+            const int u = base + lane;
+            const int c = u < kTileUnits ? cnt[u] : 0;
+            int incl = c;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, d);
+                if (lane >= d) incl += v;
             }
-            if (lane == 0) cnt[3 * k + c] = n;
+            if (u < kTileUnits) ustart[u] = run + incl - c;
+            run += __shfl_sync(0xffffffffu, incl, 31);
         }
+        if (lane == 0) ustart[kTileUnits] = run;
     }
     __syncthreads();
 
-    JobIter it_jobs{cnt, t_eff, p.kvol, L::kNAlign, 0, 0, 0};
+    JobIter it_jobs{ustart, t_eff, p.kvol, L::kNAlign, (int)((blockIdx.x * 11u + blockIdx.y * 5u) % (kVol3 - 1)),
+                    0, 0, 0, 0, 0};
     Job job;
     bool aborted = false;
 
@@ -292,7 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = 0; c < nchunks; ++c, ++it) {
                     const int s = it % S;
                     const uint32_t ph = (uint32_t)(it / S) & 1u;
-                    if (!wait_bar(empty0 + 8 * s, ph ^ 1u, abort_flag, p.err)) {
+                    if (!wait_bar<true>(empty0 + 8 * s, ph ^ 1u, abort_flag, p.err)) {
                         aborted = true;
                         break;
                     }
@@ -318,7 +338,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         aborted = true;
                         break;
                     }
-                    tc_fence_after();
                 }
                 const uint32_t idesc = idesc_bf16(BM, (uint32_t)job.ncols);
                 for (int c = 0; c < nchunks; ++c, ++it) {
@@ -328,8 +347,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         aborted = true;
                         break;
                     }
-                    tc_fence_after();
-                    fence_proxy_async_smem();
                     const uint32_t a_base = smem_addr(stages + s * L::kStageBytes);
                     const uint32_t b_base = a_base + L::kAPad;
 #pragma unroll
@@ -357,38 +374,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp < kWarpFold0) {
         // ------------------------------------------------ gather producers
+        // Per job: resolve this thread's source rows once (independent smem
+        // lookups), then issue the 16-byte copies of every input-channel chunk.
+        // Each thread arrives on the stage barrier when its own copies land
+        // (cp.async.mbarrier.arrive.noinc), so no producer ever waits for data.
+        constexpr int kMaxPass = kCentreCols / L::kRowsPerPass;
         const int g = threadIdx.x - kWarpGather0 * 32;
+        GroupWait gwait{3, kGatherThreads, g == 0, wait_slots, 0};
         const int q = g % L::kThreadsPerRow;
         const int prow = g / L::kThreadsPerRow;
         int it = 0;
         it_jobs.start();
         while (!aborted && it_jobs.next(job)) {
+            const __nv_bfloat16* src[kMaxPass];
+            uint32_t bytes[kMaxPass];
+            uint32_t dst_off[kMaxPass];
+#pragma unroll
+            for (int ps = 0; ps < kMaxPass; ++ps) {
+                const int pr = prow + ps * L::kRowsPerPass;
+                int64_t j = 0;
+                bytes[ps] = 0;
+                if (pr < job.n) {
+                    j = job.centre ? row0 + job.first + pr : (int64_t)pj_s[job.base + job.first + pr];
+                    bytes[ps] = 16;
+                }
+                src[ps] = p.x + j * p.cin + q * 8;
+                const uint32_t lin = (uint32_t)(pr * L::kRowBytes + q * 16);
+                dst_off[ps] = lin ^ (((lin >> 7) & L::kSwizzleMask) << 4);
+            }
+            const int npass = (job.ncols - prow + L::kRowsPerPass - 1) / L::kRowsPerPass;
             for (int c = 0; c < nchunks; ++c, ++it) {
                 const int s = it % S;
                 const uint32_t ph = (uint32_t)(it / S) & 1u;
-                if (!warp_wait_bar(empty0 + 8 * s, ph ^ 1u, abort_flag, p.err)) {
+                if (!gwait(empty0 + 8 * s, ph ^ 1u, abort_flag, p.err)) {
                     aborted = true;
                     break;
                 }
                 const uint32_t b_base = smem_addr(stages + s * L::kStageBytes) + L::kAPad;
-                const int col_off = c * KC + q * 8;
-                for (int pr = prow; pr < job.ncols; pr += L::kRowsPerPass) {
-                    const __nv_bfloat16* src = p.x;
-                    uint32_t bytes = 0;
-                    if (pr < job.n) {
-                        int64_t j;
-                        if (job.centre) {
-                            j = row0 + job.first + pr;
-                        } else {
-                            const int r = list_row(lists, cnt, job.k, job.first + pr);
-                            j = nbr_s[r * kVol3 + job.k];
-                        }
-                        src = p.x + j * p.cin + col_off;
-                        bytes = 16;
-                    }
-                    const uint32_t lin = (uint32_t)(pr * L::kRowBytes + q * 16);
-                    cp_async_16(b_base + (lin ^ (((lin >> 7) & L::kSwizzleMask) << 4)), src, bytes);
-                }
+#pragma unroll
+                for (int ps = 0; ps < kMaxPass; ++ps)
+                    if (ps < npass) cp_async_16(b_base + dst_off[ps], src[ps] + c * KC, bytes[ps]);
                 cp_async_mbar_arrive_noinc(full0 + 8 * s);
             }
         }
@@ -400,57 +425,59 @@ __global__ void __launch_bounds__(kThreads, 1)
         // one warp per lane quarter.
         const int quarter = warp & 3;
         const int sub = (warp - kWarpFold0) >> 2;
+        GroupWait fwait{2, 32 * kFoldWarps, threadIdx.x == kWarpFold0 * 32, wait_slots + 2, 0};
         const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
         int sj = 0;
         it_jobs.start();
         while (!aborted && it_jobs.next(job)) {
             if (job.centre) continue;
             const int b = sj & 1;
-            if (!warp_wait_bar(sfull0 + 8 * b, (uint32_t)(sj >> 1) & 1u, abort_flag, p.err)) {
+            if (!fwait(sfull0 + 8 * b, (uint32_t)(sj >> 1) & 1u, abort_flag, p.err)) {
                 aborted = true;
                 break;
             }
-            tc_fence_after();
             const uint32_t scr = tmem + lane_base + kScratchCol0 + (uint32_t)b * kScratchCols;
-            const int k = job.k;
-            const int cls_start = (sub >= 1 ? cnt[3 * k] : 0) + (sub >= 2 ? cnt[3 * k + 1] : 0);
-            const int lo = max(job.first, cls_start);
-            const int hi = min(job.first + job.n, cls_start + cnt[3 * k + sub]);
-            const uint16_t* lst = lists + (3 * k + sub) * kClassRows;
-            bool released = false;
-            for (int g0 = lo; g0 < hi; g0 += kFoldGroup) {
-                float v[kFoldGroup], a[kFoldGroup];
-                uint32_t col[kFoldGroup];
-                tmem_ld_x16(scr + (uint32_t)(g0 - job.first), v);
-                if (g0 == lo) tmem_wait_st();  // this warp's stores of the previous job have landed
+            // this warp's class of the job's offset: flat entries [cls_lo, cls_hi)
+            const int cls_lo = ustart[3 * job.ks + sub] - job.base, cls_hi = ustart[3 * job.ks + sub + 1] - job.base;
+            const int lo = max(job.first, cls_lo);
+            const int hi = min(job.first + job.n, cls_hi);
+            const uint16_t* lst = pr_s + job.base;
+            // 1) read this warp's scratch columns with wide loads and hand the
+            //    buffer back to the MMA issuer at once;
+            float v[kScratchCols];
+            const int ng = (hi - lo + kFoldGroup - 1) / kFoldGroup;  // <= 3
+            if (ng > 0) tmem_ld_x16(scr + (uint32_t)(lo - job.first), v);
+            if (ng > 1) tmem_ld_x16(scr + (uint32_t)(lo - job.first + kFoldGroup), v + kFoldGroup);
+            if (ng > 2) tmem_ld_x16(scr + (uint32_t)(lo - job.first + 2 * kFoldGroup), v + 2 * kFoldGroup);
+            tmem_wait_ld();  // the scratch values are in registers
+            __syncwarp();
+            if (lane == 0) mbar_arrive(sempty0 + 8 * b);
+            // 2) then add them into the accumulator columns of their rows.
+            if (ng > 0) tmem_wait_st();  // this warp's stores of the previous job have landed
 #pragma unroll
-                for (int i = 0; i < kFoldGroup; ++i) {
-                    const int e = g0 + i;
-                    const uint32_t r = lst[min(e, hi - 1) - cls_start];
-                    col[i] = tmem + lane_base + (e < hi ? r : kDummyCol0 + (uint32_t)i);
-                    tmem_ld_x1(col[i], a[i]);
-                }
-                tmem_wait_ld();
-                if (g0 + kFoldGroup >= hi) {  // last group: the scratch buffer has been read
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(sempty0 + 8 * b);
-                    released = true;
-                }
+            for (int gi = 0; gi < kScratchCols / kFoldGroup; ++gi) {
+                if (gi < ng) {
+                    const int g0 = lo + gi * kFoldGroup;
+                    float a[kFoldGroup];
+                    uint32_t col[kFoldGroup];
 #pragma unroll
-                for (int i = 0; i < kFoldGroup; ++i) tmem_st_x1(col[i], a[i] + v[i]);
-            }
-            if (!released) {
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(sempty0 + 8 * b);
+                    for (int i = 0; i < kFoldGroup; ++i) {
+                        const int e = g0 + i;
+                        const uint32_t r = lst[min(e, hi - 1)];
+                        col[i] = tmem + lane_base + (e < hi ? r : kDummyCol0 + (uint32_t)i);
+                        tmem_ld_x1(col[i], a[i]);
+                    }
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < kFoldGroup; ++i) tmem_st_x1(col[i], a[i] + v[gi * kFoldGroup + i]);
+                }
             }
             ++sj;
         }
         tmem_wait_st();
         tc_fence_before();
         named_barrier(1, 32 * kFoldWarps);  // every fold store has landed before any epilogue read
-        if (!aborted && warp_wait_bar(accfull, 0, abort_flag, p.err)) {
+        if (!aborted && fwait(accfull, 0, abort_flag, p.err)) {
             tc_fence_after();
             const bool lane_ok = lane < L::kChPerWarp;
             const int ch_base = cblk * BM + quarter * L::kChPerWarp;
@@ -544,7 +571,10 @@ spconv_status_t launch(const MapData& m, const void* x, int cin, const void* w, 
         return SPCONV_ERR_CUDA;
     }
     Params p;
-    p.nbr = m.nbr;
+    p.tile_counts = m.tile_counts;
+    p.tile_off = m.tile_off;
+    p.pair_r = m.pair_r;
+    p.pair_j = m.pair_j;
     p.n = m.n;
     p.kvol = kvol;
     p.x = static_cast<const __nv_bfloat16*>(x);

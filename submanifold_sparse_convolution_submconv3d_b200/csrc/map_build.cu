@@ -119,3 +119,149 @@ cudaError_t launch_build_map(const int32_t* coords, int64_t n, const int32_t ext
 }
 
 }  // namespace spconv
+
+// ---------------------------------------------------------------------------
+// Tile metadata.  One CTA per tile stages the tile's [rows, 27] map rows in
+// shared memory (coalesced), then warps scan the (offset, class) units with
+// ballots: k_tile_count writes the per-unit counts and the tile's padded entry
+// total; k_tile_scan turns the totals into offsets; k_tile_fill writes the
+// entries (local row, neighbour row) in unit order, rows ascending per unit.
+namespace spconv {
+namespace {
+
+constexpr int kMetaThreads = 256;
+
+__device__ __forceinline__ void stage_tile_rows(const int32_t* __restrict__ nbr, int64_t row0, int t_eff,
+                                                int32_t* __restrict__ tile_s) {
+    const int words = t_eff * kVol3;
+    const int32_t* src = nbr + row0 * kVol3;
+    for (int i = threadIdx.x; i < words; i += blockDim.x) tile_s[i] = __ldg(src + i);
+}
+
+__device__ __forceinline__ int unit_offset(int u) {
+    const int ks = u / kTileClasses;
+    return ks < kCentre ? ks : ks + 1;
+}
+
+__global__ void k_tile_count(const int32_t* __restrict__ nbr, int64_t n, int32_t* __restrict__ tile_counts,
+                             int64_t* __restrict__ tile_total) {
+    __shared__ int32_t tile_s[kTileRows * kVol3];
+    __shared__ int32_t cnt_s[kTileUnits];
+    const int64_t t = blockIdx.x;
+    const int64_t row0 = t * kTileRows;
+    const int t_eff = (int)min((int64_t)kTileRows, n - row0);
+    stage_tile_rows(nbr, row0, t_eff, tile_s);
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int u = warp; u < kTileUnits; u += kMetaThreads / 32) {
+        const int k = unit_offset(u), c = u % kTileClasses;
+        int count = 0;
+        for (int base = 0; base < kTileRows / kTileClasses; base += 32) {
+            const int r = c + kTileClasses * (base + lane);
+            const bool hit = r < t_eff && tile_s[r * kVol3 + k] >= 0;
+            count += __popc(__ballot_sync(0xffffffffu, hit));
+        }
+        if (lane == 0) cnt_s[u] = count;
+    }
+    __syncthreads();
+    if (threadIdx.x < kTileCountStride)
+        tile_counts[t * kTileCountStride + threadIdx.x] = threadIdx.x < kTileUnits ? cnt_s[threadIdx.x] : 0;
+    if (threadIdx.x == 0) {
+        int64_t total = 0;
+        for (int u = 0; u < kTileUnits; ++u) total += cnt_s[u];
+        tile_total[t] = (total + kTileEntryAlign - 1) / kTileEntryAlign * kTileEntryAlign;
+    }
+}
+
+// Exclusive scan of the per-tile totals (in place, one CTA): off[t] = sum of
+// totals before t; off[ntiles] = grand total.
+__global__ void k_tile_scan(int64_t* __restrict__ off, int64_t ntiles) {
+    __shared__ int64_t part[1024];
+    const int64_t per = (ntiles + blockDim.x - 1) / blockDim.x;
+    const int64_t lo = threadIdx.x * per, hi = min(ntiles, lo + per);
+    int64_t sum = 0;
+    for (int64_t i = lo; i < hi; ++i) sum += off[i];
+    part[threadIdx.x] = sum;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int64_t run = 0;
+        for (int i = 0; i < (int)blockDim.x; ++i) {
+            const int64_t v = part[i];
+            part[i] = run;
+            run += v;
+        }
+        off[ntiles] = run;
+    }
+    __syncthreads();
+    int64_t run = part[threadIdx.x];
+    for (int64_t i = lo; i < hi; ++i) {
+        const int64_t v = off[i];
+        off[i] = run;
+        run += v;
+    }
+}
+
+__global__ void k_tile_fill(const int32_t* __restrict__ nbr, int64_t n, const int32_t* __restrict__ tile_counts,
+                            const int64_t* __restrict__ tile_off, uint16_t* __restrict__ pair_r,
+                            int32_t* __restrict__ pair_j) {
+    __shared__ int32_t tile_s[kTileRows * kVol3];
+    __shared__ int32_t start_s[kTileUnits];
+    const int64_t t = blockIdx.x;
+    const int64_t row0 = t * kTileRows;
+    const int t_eff = (int)min((int64_t)kTileRows, n - row0);
+    stage_tile_rows(nbr, row0, t_eff, tile_s);
+    if (threadIdx.x == 0) {
+        int run = 0;
+        for (int u = 0; u < kTileUnits; ++u) {
+            start_s[u] = run;
+            run += tile_counts[t * kTileCountStride + u];
+        }
+        // zero the padding entries of this tile
+        const int64_t end = tile_off[t + 1];
+        for (int64_t e = tile_off[t] + run; e < end; ++e) {
+            pair_r[e] = 0;
+            pair_j[e] = 0;
+        }
+    }
+    __syncthreads();
+    const int64_t base = tile_off[t];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int u = warp; u < kTileUnits; u += kMetaThreads / 32) {
+        const int k = unit_offset(u), c = u % kTileClasses;
+        int pos = start_s[u];
+        for (int b = 0; b < kTileRows / kTileClasses; b += 32) {
+            const int r = c + kTileClasses * (b + lane);
+            const int32_t j = r < t_eff ? tile_s[r * kVol3 + k] : -1;
+            const unsigned m = __ballot_sync(0xffffffffu, j >= 0);
+            if (j >= 0) {
+                const int64_t e = base + pos + __popc(m & ((1u << lane) - 1u));
+                pair_r[e] = (uint16_t)r;
+                pair_j[e] = j;
+            }
+            pos += __popc(m);
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_tile_count(const int32_t* nbr, int64_t n, int32_t* tile_counts, int64_t* tile_off,
+                              cudaStream_t stream) {
+    const int64_t nt = num_tiles(n);
+    if (nt == 0) return cudaMemsetAsync(tile_off, 0, sizeof(int64_t), stream);
+    k_tile_count<<<(unsigned)nt, kMetaThreads, 0, stream>>>(nbr, n, tile_counts, tile_off);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    k_tile_scan<<<1, 1024, 0, stream>>>(tile_off, nt);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_tile_fill(const int32_t* nbr, int64_t n, const int32_t* tile_counts, const int64_t* tile_off,
+                             uint16_t* pair_r, int32_t* pair_j, cudaStream_t stream) {
+    const int64_t nt = num_tiles(n);
+    if (nt == 0) return cudaSuccess;
+    k_tile_fill<<<(unsigned)nt, kMetaThreads, 0, stream>>>(nbr, n, tile_counts, tile_off, pair_r, pair_j);
+    return cudaGetLastError();
+}
+
+}  // namespace spconv

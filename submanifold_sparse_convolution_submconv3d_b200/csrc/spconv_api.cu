@@ -78,10 +78,29 @@ spconv_status_t spconv_build_map(const int32_t* coords, int64_t n, const int32_t
     e = cudaMalloc(&table, slots * 16);
     if (e == cudaSuccess) e = cudaMalloc(&flags, sizeof(spconv::BuildFlags));
     if (e == cudaSuccess && kernel_size == 3 && n > 0) e = cudaMalloc(&m->d.nbr, (size_t)n * spconv::kVol3 * sizeof(int32_t));
+    const int64_t ntiles = spconv::num_tiles(n);
+    const bool tiles = kernel_size == 3 && n > 0;
+    if (e == cudaSuccess && tiles) e = cudaMalloc(&m->d.tile_counts, (size_t)ntiles * spconv::kTileCountStride * 4);
+    if (e == cudaSuccess && tiles) e = cudaMalloc(&m->d.tile_off, (size_t)(ntiles + 1) * sizeof(int64_t));
     if (e == cudaSuccess)
         e = spconv::launch_build_map(coords, n, extent, kernel_size, table, slots, m->d.nbr, flags, stream);
+    if (e == cudaSuccess && tiles) e = spconv::launch_tile_count(m->d.nbr, n, m->d.tile_counts, m->d.tile_off, stream);
+    int64_t total_entries = 0;
+    if (e == cudaSuccess && tiles)
+        e = cudaMemcpyAsync(&total_entries, m->d.tile_off + ntiles, sizeof(int64_t), cudaMemcpyDeviceToHost, stream);
     if (e == cudaSuccess) e = cudaMemcpyAsync(&host_flags, flags, sizeof(host_flags), cudaMemcpyDeviceToHost, stream);
     if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    // Second phase (only if the map is valid): entry arrays of the tile metadata.
+    if (e == cudaSuccess && tiles && host_flags.err == 0) {
+        m->d.tile_entries = total_entries;
+        const size_t ne = total_entries > 0 ? (size_t)total_entries : 1;
+        e = cudaMalloc(&m->d.pair_r, ne * sizeof(uint16_t));
+        if (e == cudaSuccess) e = cudaMalloc(&m->d.pair_j, ne * sizeof(int32_t));
+        if (e == cudaSuccess)
+            e = spconv::launch_tile_fill(m->d.nbr, n, m->d.tile_counts, m->d.tile_off, m->d.pair_r, m->d.pair_j,
+                                         stream);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    }
     if (e != cudaSuccess) {
         status = fail_cuda(e, "spconv_build_map");
     } else if (host_flags.err & spconv::kErrCoordRange) {
@@ -94,9 +113,7 @@ spconv_status_t spconv_build_map(const int32_t* coords, int64_t n, const int32_t
     cudaFree(table);
     cudaFree(flags);
     if (status != SPCONV_OK) {
-        cudaFree(m->d.nbr);
-        cudaFree(m->d.fwd_err);
-        delete m;
+        spconv_free(m);
         return status;
     }
     m->d.pairs = kernel_size == 3 ? (int64_t)host_flags.pairs : n;
@@ -108,6 +125,10 @@ spconv_status_t spconv_free(spconv_map_t map) {
     if (!map) return SPCONV_OK;
     cudaFree(map->d.nbr);
     cudaFree(map->d.fwd_err);
+    cudaFree(map->d.tile_counts);
+    cudaFree(map->d.tile_off);
+    cudaFree(map->d.pair_r);
+    cudaFree(map->d.pair_j);
     delete map;
     return SPCONV_OK;
 }
