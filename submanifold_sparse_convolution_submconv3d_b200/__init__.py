@@ -56,7 +56,19 @@ def _load() -> ctypes.CDLL:
     return lib
 
 
-lib = _load()
+try:
+    lib = _load()
+    _LOAD_ERROR = None
+except (OSError, AttributeError, ImportError) as _exc:  # missing or stale library
+    lib = None
+    _LOAD_ERROR = _exc
+
+
+def _require() -> None:
+    """Raise if the CUDA library could not be loaded: there is no fallback path."""
+    if lib is None:
+        raise ImportError(f"the CUDA library {LIB_PATH} is unavailable ({_LOAD_ERROR}); build it with "
+                          "python -m submanifold_sparse_convolution_submconv3d_b200.build")
 
 
 def _check(status: int) -> None:
@@ -112,6 +124,7 @@ class SubmMap:
 
 def spconv_build_map(coords: torch.Tensor, extent, kernel_size: int = 3, stream=None) -> SubmMap:
     """Build the neighbour map of int32 [N, 4] (b, x, y, z) CUDA coordinates."""
+    _require()
     if coords.dtype != torch.int32 or not coords.is_cuda or coords.dim() != 2 or coords.shape[1] != 4:
         raise ValueError("coords must be a CUDA int32 tensor of shape [N, 4]")
     coords = coords.contiguous()
@@ -126,6 +139,7 @@ def spconv_build_map(coords: torch.Tensor, extent, kernel_size: int = 3, stream=
 def spconv_subm_forward(m: SubmMap, x: torch.Tensor, w: torch.Tensor, bias: torch.Tensor | None = None,
                         out: torch.Tensor | None = None, algo: int = ALGO_AUTO, stream=None) -> torch.Tensor:
     """One SubMConv3d layer: x [N, Cin], w [K^3, Cin, Cout], bias [Cout] -> out [N, Cout]."""
+    _require()
     if x.dtype not in _DTYPES:
         raise ValueError("x must be float32 or bfloat16")
     for t in (w,) + (() if bias is None else (bias,)):
@@ -154,6 +168,7 @@ def spconv_free(m: SubmMap) -> None:
 
 
 def spconv_debug_set_table_slots(slots: int) -> None:
+    _require()
     _check(lib.spconv_debug_set_table_slots(int(slots)))
 
 
