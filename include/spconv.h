@@ -155,6 +155,35 @@ SPCONV_API spconv_status_t spconv_subm_forward_algo(spconv_map_t map, spconv_dty
  */
 SPCONV_API spconv_status_t spconv_debug_set_table_slots(int64_t slots);
 
+/*
+ * Neighbour-map build that allocates no device memory.  The pages have no
+ * counterpart: this is an interface for callers that cannot call cudaMalloc or
+ * cudaFree -- code running while another component owns the device memory (a
+ * framework's caching allocator, an arena reserved up front) and latency-critical
+ * loops, since cudaFree synchronises the whole device and cudaMalloc can stall
+ * other streams.
+ *
+ *   coords     device int32 [n, 4] (b, x, y, z), 16-byte aligned.
+ *   n          0 <= n <= 524288 (larger sets: SPCONV_ERR_UNSUPPORTED; use spconv_build_map).
+ *   extent     host int32 [3], each in [1, 65535].
+ *   nbr_out    device int32 [n, 27], caller-owned: nbr_out[i*27 + k] = row of the
+ *              active voxel at p_i + d_k, or -1 (same values as the map that
+ *              spconv_build_map builds with kernel size 3).
+ *   pairs_out  host; receives the number of entries >= 0 of nbr_out (may be NULL).
+ *   stream     stream on which the build runs; the call synchronises it once.
+ *
+ * The hash table and error flags live in one static device array of 16 MiB plus
+ * 256 bytes that every GPU loading this library holds until the process exits.
+ * The first call on a device looks up that array's device address (with the
+ * device current); make that first call before any stream capture.  Every call
+ * shares the array and clears it before use, so calls that overlap on the GPU
+ * (on different streams or host threads) race and must not be issued.  Errors:
+ * as spconv_build_map, plus SPCONV_ERR_UNSUPPORTED above the size limit;
+ * spconv_last_error() describes them.
+ */
+SPCONV_API spconv_status_t spconv_build_neighbor_map_noalloc(const int32_t* coords, int64_t n, const int32_t* extent,
+                                                             int32_t* nbr_out, int64_t* pairs_out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -26,7 +26,8 @@ ALGO_AUTO, ALGO_SIMT, ALGO_TCGEN05 = 0, 1, 2
 _DTYPES = {torch.float32: 0, torch.bfloat16: 1}
 
 EXPORTED = ("spconv_build_map", "spconv_subm_forward", "spconv_free", "spconv_map_info", "spconv_map_check",
-            "spconv_last_error", "spconv_subm_forward_algo", "spconv_debug_set_table_slots")
+            "spconv_last_error", "spconv_subm_forward_algo", "spconv_debug_set_table_slots",
+            "spconv_build_neighbor_map_noalloc")
 
 
 class SpconvError(RuntimeError):
@@ -49,9 +50,11 @@ def _load() -> ctypes.CDLL:
                                     ctypes.POINTER(vp)]
     lib.spconv_map_check.argtypes = [vp, vp]
     lib.spconv_debug_set_table_slots.argtypes = [i64]
+    lib.spconv_build_neighbor_map_noalloc.argtypes = [vp, i64, vp, vp, ctypes.POINTER(i64), vp]
     lib.spconv_last_error.restype = ctypes.c_char_p
     for name in ("spconv_build_map", "spconv_subm_forward", "spconv_subm_forward_algo", "spconv_free",
-                 "spconv_map_info", "spconv_map_check", "spconv_debug_set_table_slots"):
+                 "spconv_map_info", "spconv_map_check", "spconv_debug_set_table_slots",
+                 "spconv_build_neighbor_map_noalloc"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -167,6 +170,30 @@ def spconv_free(m: SubmMap) -> None:
     m.free()
 
 
+def spconv_build_neighbor_map_noalloc(coords: torch.Tensor, extent, out: torch.Tensor | None = None,
+                                      stream=None) -> tuple[torch.Tensor, int]:
+    """Dense int32 [N, 27] neighbour map built without any device allocation by
+    the library (scratch in a static device array; N <= 524288).  The caller may
+    pass ``out``; otherwise the binding allocates it with torch before the call.
+    Returns (map, pairs)."""
+    _require()
+    if coords.dtype != torch.int32 or not coords.is_cuda or coords.dim() != 2 or coords.shape[1] != 4:
+        raise ValueError("coords must be a CUDA int32 tensor of shape [N, 4]")
+    coords = coords.contiguous()
+    n = coords.shape[0]
+    if out is None:
+        out = torch.empty((n, 27), dtype=torch.int32, device=coords.device)
+    elif out.shape != (n, 27) or out.dtype != torch.int32 or not out.is_contiguous():
+        raise ValueError("out must be a contiguous int32 [N, 27] tensor")
+    ext = (ctypes.c_int32 * 3)(*[int(v) for v in extent])
+    pairs = ctypes.c_int64()
+    with torch.cuda.device(coords.device):
+        _check(lib.spconv_build_neighbor_map_noalloc(coords.data_ptr() if n else None, n, ext,
+                                                     out.data_ptr() if n else None, ctypes.byref(pairs),
+                                                     _stream(stream)))
+    return out, pairs.value
+
+
 def spconv_debug_set_table_slots(slots: int) -> None:
     _require()
     _check(lib.spconv_debug_set_table_slots(int(slots)))
@@ -174,5 +201,5 @@ def spconv_debug_set_table_slots(slots: int) -> None:
 
 __all__ = ["OK", "INVALID_ARG", "UNSUPPORTED", "COORD_RANGE", "DUPLICATE", "TABLE_FULL", "OOM", "CUDA_ERROR",
            "TIMEOUT", "SubmMap", "SpconvError", "spconv_build_map", "spconv_subm_forward", "spconv_free",
-           "spconv_debug_set_table_slots", "lib", "LIB_PATH", "EXPORTED",
+           "spconv_debug_set_table_slots", "spconv_build_neighbor_map_noalloc", "lib", "LIB_PATH", "EXPORTED",
            "ALGO_AUTO", "ALGO_SIMT", "ALGO_TCGEN05"]

@@ -5,6 +5,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <string>
+
 #include "spconv.h"
 
 namespace spconv {
@@ -63,6 +65,9 @@ struct MapData {
     int device = 0;
     int num_sms = 0;
 };
+
+// Sets the calling thread's message returned by spconv_last_error().
+void set_last_error(const std::string& msg);
 
 // Launchers (each returns cudaSuccess or the first CUDA error).
 cudaError_t launch_build_map(const int32_t* coords, int64_t n, const int32_t extent[3], int32_t kernel_size,

@@ -33,6 +33,10 @@ uint64_t next_pow2(uint64_t v) {
 
 }  // namespace
 
+namespace spconv {
+void set_last_error(const std::string& msg) { g_last_error = msg; }
+}  // namespace spconv
+
 extern "C" {
 
 const char* spconv_last_error(void) { return g_last_error.c_str(); }
