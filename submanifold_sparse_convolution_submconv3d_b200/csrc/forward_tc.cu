@@ -45,7 +45,8 @@ using namespace sm100;
 constexpr int kClasses = kTileClasses;           // rows split by r % 3 between fold warps
 constexpr int kMaxEntries = (kVol3 - 1) * kTileRows;  // tile metadata entries, worst case
 constexpr int kScratchCols = 48;
-constexpr int kCentreCols = 128;
+constexpr int kCentreCols = 48;   // centre jobs: 48-row slices straight into the accumulator
+constexpr int kJobRows = 48;      // rows of one job's B tile (centre slice or compacted offset part)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kScratchCol0 = kTileRows;      // scratch buffer b at column 384 + 48 b
 constexpr uint32_t kDummyCol0 = kScratchCol0 + 2 * kScratchCols;  // 480..495: fold padding targets
@@ -62,16 +63,24 @@ __host__ __device__ constexpr int round_up(int v, int m) { return (v + m - 1) / 
 // Shared-memory carve-up, identical on host and device.
 template <int BM, int KC>
 struct Layout {
+    // B tile: kJobRows gathered rows x KC channels, K-major, split into swizzle
+    // atoms of up to 64 channels (128 bytes) each: [atom][row][atom row bytes].
+    static constexpr int kAtomElems = KC >= 64 ? 64 : KC;
+    static constexpr int kAtoms = KC / kAtomElems;
+    static constexpr int kAtomRowBytes = kAtomElems * 2;
+    static constexpr int kBAtomBytes = kJobRows * kAtomRowBytes;  // 1024-multiple when kAtoms > 1
     static constexpr int kRowBytes = KC * 2;                      // one gathered row chunk
     static constexpr int kThreadsPerRow = kRowBytes / 16;
     static constexpr int kRowsPerPass = kGatherThreads / kThreadsPerRow;
-    static constexpr uint32_t kSwizzleMask = kRowBytes / 16 - 1;
+    static constexpr int kChunksPerAtom = kAtomRowBytes / 16;
+    static constexpr uint32_t kSwizzleMask = kAtomRowBytes / 16 - 1;
     static constexpr int kABytes = BM * KC * 2;                   // weight tile per stage
     static constexpr int kAPad = round_up(kABytes, 1024);
-    static constexpr int kBPad = round_up(kCentreCols * kRowBytes, 1024);  // up to 128 gathered rows
+    static constexpr int kBPad = round_up(kAtoms * kBAtomBytes, 1024);
     static constexpr int kStageBytes = kAPad + kBPad;
-    static constexpr uint32_t kBLayout = KC == 64 ? 2u : (KC == 32 ? 4u : 6u);  // 128/64/32-byte swizzle
-    static constexpr uint32_t kBSbo = 8 * kRowBytes;
+    static constexpr uint32_t kBLayout = kAtomRowBytes == 128 ? 2u : (kAtomRowBytes == 64 ? 4u : 6u);
+    static constexpr uint32_t kBSbo = 8 * kAtomRowBytes;
+    static_assert(kAtoms == 1 || kBAtomBytes % 1024 == 0, "B atoms must keep the swizzle alignment");
     static constexpr int kNAlign = BM == 128 ? 16 : 8;
     static constexpr int kChPerWarp = BM / 4;                     // channels of one TMEM lane quarter
 
@@ -245,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- set-up: barriers, TMEM, neighbour rows of the tile (cp.async, 16 B)
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(full0 + 8 * s, 1 + kGatherThreads);
+            mbar_init(full0 + 8 * s, 1 + kGatherThreads);  // weight TMA + every gather thread
             mbar_init(empty0 + 8 * s, 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -311,8 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             while (!aborted && it_jobs.next(job)) {
                 for (int c = 0; c < nchunks; ++c, ++it) {
                     const int s = it % S;
-                    const uint32_t ph = (uint32_t)(it / S) & 1u;
-                    if (!wait_bar<true>(empty0 + 8 * s, ph ^ 1u, abort_flag, p.err)) {
+                    if (!wait_bar<true>(empty0 + 8 * s, ((uint32_t)(it / S) & 1u) ^ 1u, abort_flag, p.err)) {
                         aborted = true;
                         break;
                     }
@@ -352,7 +360,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int kk = 0; kk < KC / 16; ++kk) {
                         const uint64_t adesc = smem_desc(a_base + kk * 2048, KC * 128, 1024, 2);
-                        const uint64_t bdesc = smem_desc(b_base + kk * 32, 16, L::kBSbo, L::kBLayout);
+                        constexpr int kStepsPerAtom = L::kAtomElems / 16;
+                        const uint64_t bdesc =
+                            smem_desc(b_base + (kk / kStepsPerAtom) * L::kBAtomBytes + (kk % kStepsPerAtom) * 32, 16,
+                                      L::kBSbo, L::kBLayout);
                         mma_bf16(d, adesc, bdesc, idesc, (c > 0 || kk > 0) ? 1u : 0u);
                     }
                     mma_commit(empty0 + 8 * s);
@@ -374,35 +385,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp < kWarpFold0) {
         // ------------------------------------------------ gather producers
-        // Per job: resolve this thread's source rows once (independent smem
-        // lookups), then issue the 16-byte copies of every input-channel chunk.
-        // Each thread arrives on the stage barrier when its own copies land
+        // The four warps fill every stage together.  Per job: resolve this
+        // thread's source rows once (independent shared-memory lookups), then
+        // issue the 16-byte copies of every input-channel chunk.  Each thread
+        // arrives on the stage barrier when its own copies land
         // (cp.async.mbarrier.arrive.noinc), so no producer ever waits for data.
-        constexpr int kMaxPass = kCentreCols / L::kRowsPerPass;
+        constexpr int kMaxPass = (kJobRows + L::kRowsPerPass - 1) / L::kRowsPerPass;
         const int g = threadIdx.x - kWarpGather0 * 32;
         GroupWait gwait{3, kGatherThreads, g == 0, wait_slots, 0};
         const int q = g % L::kThreadsPerRow;
         const int prow = g / L::kThreadsPerRow;
+        const int atom = q / L::kChunksPerAtom, qa = q % L::kChunksPerAtom;
         int it = 0;
         it_jobs.start();
         while (!aborted && it_jobs.next(job)) {
-            const __nv_bfloat16* src[kMaxPass];
-            uint32_t bytes[kMaxPass];
+            int64_t src_row[kMaxPass];
             uint32_t dst_off[kMaxPass];
 #pragma unroll
             for (int ps = 0; ps < kMaxPass; ++ps) {
                 const int pr = prow + ps * L::kRowsPerPass;
-                int64_t j = 0;
-                bytes[ps] = 0;
-                if (pr < job.n) {
-                    j = job.centre ? row0 + job.first + pr : (int64_t)pj_s[job.base + job.first + pr];
-                    bytes[ps] = 16;
-                }
-                src[ps] = p.x + j * p.cin + q * 8;
-                const uint32_t lin = (uint32_t)(pr * L::kRowBytes + q * 16);
-                dst_off[ps] = lin ^ (((lin >> 7) & L::kSwizzleMask) << 4);
+                src_row[ps] = -1;
+                if (pr < job.n) src_row[ps] = job.centre ? row0 + job.first + pr : (int64_t)pj_s[job.base + job.first + pr];
+                const uint32_t lin = (uint32_t)(pr * L::kAtomRowBytes + qa * 16);
+                dst_off[ps] = (uint32_t)(atom * L::kBAtomBytes) + (lin ^ (((lin >> 7) & L::kSwizzleMask) << 4));
             }
-            const int npass = (job.ncols - prow + L::kRowsPerPass - 1) / L::kRowsPerPass;
             for (int c = 0; c < nchunks; ++c, ++it) {
                 const int s = it % S;
                 const uint32_t ph = (uint32_t)(it / S) & 1u;
@@ -412,8 +418,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const uint32_t b_base = smem_addr(stages + s * L::kStageBytes) + L::kAPad;
 #pragma unroll
-                for (int ps = 0; ps < kMaxPass; ++ps)
-                    if (ps < npass) cp_async_16(b_base + dst_off[ps], src[ps] + c * KC, bytes[ps]);
+                for (int ps = 0; ps < kMaxPass; ++ps) {
+                    const int pr = prow + ps * L::kRowsPerPass;
+                    if (pr < job.ncols) {
+                        const bool hit = src_row[ps] >= 0;
+                        cp_async_16(b_base + dst_off[ps], p.x + (hit ? src_row[ps] : 0) * p.cin + c * KC + q * 8,
+                                    hit ? 16u : 0u);
+                    }
+                }
                 cp_async_mbar_arrive_noinc(full0 + 8 * s);
             }
         }
@@ -598,12 +610,14 @@ spconv_status_t launch_forward_tcgen05(const MapData& m, const void* x, int cin,
     if (cin % 16 != 0 || cout % 64 != 0) return SPCONV_ERR_UNSUPPORTED;
     if (m.n == 0) return SPCONV_OK;
     const bool bm128 = cout % 128 == 0;
-    const int kc = cin % 64 == 0 ? 64 : (cin % 32 == 0 ? 32 : 16);
+    const int kc = cin % 128 == 0 ? 128 : (cin % 64 == 0 ? 64 : (cin % 32 == 0 ? 32 : 16));
     if (bm128) {
+        if (kc == 128) return launch<128, 128>(m, x, cin, w, bias, out, cout, stream, ce);
         if (kc == 64) return launch<128, 64>(m, x, cin, w, bias, out, cout, stream, ce);
         if (kc == 32) return launch<128, 32>(m, x, cin, w, bias, out, cout, stream, ce);
         return launch<128, 16>(m, x, cin, w, bias, out, cout, stream, ce);
     }
+    if (kc == 128) return launch<64, 128>(m, x, cin, w, bias, out, cout, stream, ce);
     if (kc == 64) return launch<64, 64>(m, x, cin, w, bias, out, cout, stream, ce);
     if (kc == 32) return launch<64, 32>(m, x, cin, w, bias, out, cout, stream, ce);
     return launch<64, 16>(m, x, cin, w, bias, out, cout, stream, ce);
