@@ -55,12 +55,14 @@ struct MapData {
     int64_t pairs = 0;
     int32_t* nbr = nullptr;        // device [n, 27] (kernel size 3), else null
     // tile metadata (kernel size 3): counts [ntiles][kTileCountStride], entry offsets
-    // [ntiles + 1] (multiples of kTileEntryAlign), local rows and neighbour rows per entry
+    // [ntiles + 1] (multiples of kTileEntryAlign; slot ntiles + 1 holds the largest
+    // tile's count), local rows and neighbour rows per entry
     int32_t* tile_counts = nullptr;
     int64_t* tile_off = nullptr;
     uint16_t* pair_r = nullptr;
     int32_t* pair_j = nullptr;
     int64_t tile_entries = 0;
+    int64_t tile_max_entries = 0;  // entries of the fullest tile (a multiple of kTileEntryAlign)
     unsigned int* fwd_err = nullptr;  // device word: forward-kernel error bits
     int device = 0;
     int num_sms = 0;

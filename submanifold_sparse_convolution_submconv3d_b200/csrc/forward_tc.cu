@@ -10,28 +10,33 @@
 // One CTA owns kTileRows consecutive output rows and one block of 64 or 128
 // output channels.  Tensor memory (TMEM, 128 lanes x 512 fp32 columns) holds
 //   * the accumulator: lane = output channel, column = output row of the tile;
-//   * two scratch buffers of kScratchCols columns and a few dummy columns.
-// The centre offset (every row is its own neighbour) is one dense MMA per 128
-// rows straight into the accumulator.  For every other offset the rows of the
-// tile that have a neighbour there are compacted into a list; their neighbour
-// feature rows are gathered (cp.async, 16 B, zero-filled holes and padding)
-// into a swizzled shared-memory tile and multiplied into a scratch buffer, and fold
-// warps then add each scratch column into the accumulator column of its row
-// (tcgen05.ld / tcgen05.st, no atomics).  Weights W_k arrive by TMA.  At the
-// end each output row is written exactly once, with bias, rounded to bf16.
+//   * two scratch buffers of kJobRows columns and 16 dummy columns.
+// Work is cut into jobs of at most kJobRows columns, listed once per tile in
+// shared memory: first the centre offset (every row is its own neighbour) in
+// 48-row slices that go straight into the accumulator, then for every other
+// offset the compacted list of tile rows that have a neighbour there.  A job's
+// neighbour feature rows are gathered (cp.async, 16 B, zero-filled padding) into
+// a swizzled shared-memory tile and multiplied into a scratch buffer; fold warps
+// then add each scratch column into the accumulator column of its row
+// (tcgen05.ld / tcgen05.st, no atomics).  W_k arrives by TMA once per offset
+// (once per job and channel chunk when Cin spans several chunks).  At the end
+// each output row is written exactly once, with bias, rounded to bf16.
 //
 // Warp roles (576 threads):
-//   warp 0      TMA producer of weight tiles (A operand)
+//   warp 0      TMA producer of weight tiles (A operand), a ring of 2-6 slots
 //   warp 1      TMEM allocator and tcgen05.mma issuer
-//   warps 2-5   gather producers of feature rows (B operand)
+//   warps 2-5   gather producers (B operand): warp w fills the jobs j with
+//               j % 4 == w into its own ring of slots, in order, so each ring is
+//               filled and drained strictly in sequence
 //   warps 6-17  scratch -> accumulator fold, then the epilogue: three warps per
 //               TMEM lane quarter, each owning the tile rows of one residue mod 3,
 //               so no accumulator column is touched by two warps of a quarter.
 //               Narrow TMEM accesses are issued without per-element branches;
 //               padding entries go to dedicated dummy columns.
-// Every spin-wait is bounded: after kWaitTimeoutNs the kernel records
-// kFwdErrTimeout in the map's error word, stops issuing work, lets copies in
-// flight land, frees its TMEM and returns.
+// Waiting threads are suspended on their mbarrier (try_wait with a time hint)
+// and take no issue slots.  Every wait is bounded: after kWaitTimeoutNs the
+// kernel records kFwdErrTimeout in the map's error word, stops issuing work,
+// lets copies in flight land, frees its TMEM and returns.
 #include <mutex>
 
 #include "common.cuh"
@@ -42,25 +47,40 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kClasses = kTileClasses;           // rows split by r % 3 between fold warps
-constexpr int kMaxEntries = (kVol3 - 1) * kTileRows;  // tile metadata entries, worst case
-constexpr int kScratchCols = 48;
-constexpr int kCentreCols = 48;   // centre jobs: 48-row slices straight into the accumulator
-constexpr int kJobRows = 48;      // rows of one job's B tile (centre slice or compacted offset part)
+constexpr int kClasses = kTileClasses;                   // rows split by r % 3 between fold warps
+constexpr int kJobRows = 48;                             // columns of one job (MMA N <= 48)
+constexpr int kMaxJobs = (kTileRows + kJobRows - 1) / kJobRows * kVol3;  // at most 8 jobs per offset
+constexpr int kScratchBufs = 2;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kScratchCol0 = kTileRows;      // scratch buffer b at column 384 + 48 b
-constexpr uint32_t kDummyCol0 = kScratchCol0 + 2 * kScratchCols;  // 480..495: fold padding targets
+constexpr uint32_t kScratchCol0 = kTileRows;             // scratch buffer b at column 384 + 48 b
+constexpr uint32_t kDummyCol0 = kScratchCol0 + kScratchBufs * kJobRows;  // 480..495: fold padding targets
+static_assert(kDummyCol0 + 16 <= kTmemCols, "accumulator, scratch buffers and dummy columns must fit TMEM");
 constexpr int kWarpTma = 0, kWarpMma = 1, kWarpGather0 = 2, kWarpFold0 = 6;
 constexpr int kGatherWarps = 4, kFoldWarps = 12;
 constexpr int kThreads = 32 * (kWarpFold0 + kFoldWarps);  // 576
-constexpr int kGatherThreads = 32 * kGatherWarps;
 constexpr int kFoldGroup = 16;
+constexpr int kMaxASlots = 6;                             // weight ring slots
+constexpr int kMaxBSlots = 8;                             // gather ring slots per gather warp
 constexpr uint64_t kWaitTimeoutNs = 4000000000ull;
+constexpr uint32_t kSuspendHintNs = 20000;
 constexpr int kMaxSmem = 232448;  // 227 KB opt-in limit per CTA on sm_100
 
 __host__ __device__ constexpr int round_up(int v, int m) { return (v + m - 1) / m * m; }
 
-// Shared-memory carve-up, identical on host and device.
+// Job record (int4): x = k | ks << 8 | centre << 16 | gather slot << 17 | slot
+// phase << 20 (slot and phase of the job's first channel chunk in its gather
+// warp's ring), y = first local row (centre) or first flat entry of the tile's
+// lists, z = valid columns n, w = MMA N.
+__device__ __forceinline__ int job_k(const int4& j) { return j.x & 0xFF; }
+__device__ __forceinline__ int job_ks(const int4& j) { return (j.x >> 8) & 0xFF; }
+__device__ __forceinline__ bool job_centre(const int4& j) { return (j.x >> 16) & 1; }
+__device__ __forceinline__ int job_bslot(const int4& j) { return (j.x >> 17) & 7; }
+__device__ __forceinline__ uint32_t job_bphase(const int4& j) { return (uint32_t)(j.x >> 20) & 1u; }
+
+// Shared-memory carve-up, identical on host and device:
+//   [weight ring][gather rings][job table][unit counts, unit starts]
+//   [neighbour rows][local rows][mbarriers][misc words]
+// The epilogue's staging buffer reuses the start of the rings once every MMA is done.
 template <int BM, int KC>
 struct Layout {
     // B tile: kJobRows gathered rows x KC channels, K-major, split into swizzle
@@ -69,32 +89,46 @@ struct Layout {
     static constexpr int kAtoms = KC / kAtomElems;
     static constexpr int kAtomRowBytes = kAtomElems * 2;
     static constexpr int kBAtomBytes = kJobRows * kAtomRowBytes;  // 1024-multiple when kAtoms > 1
-    static constexpr int kRowBytes = KC * 2;                      // one gathered row chunk
-    static constexpr int kThreadsPerRow = kRowBytes / 16;
-    static constexpr int kRowsPerPass = kGatherThreads / kThreadsPerRow;
+    static constexpr int kThreadsPerRow = KC * 2 / 16;            // 16-byte chunks of one row chunk
+    static constexpr int kWarpRows = 32 / kThreadsPerRow;         // rows one warp instruction covers
+    static constexpr int kPasses = kJobRows / kWarpRows;
     static constexpr int kChunksPerAtom = kAtomRowBytes / 16;
     static constexpr uint32_t kSwizzleMask = kAtomRowBytes / 16 - 1;
-    static constexpr int kABytes = BM * KC * 2;                   // weight tile per stage
+    static constexpr int kABytes = BM * KC * 2;                   // weight tile per slot
     static constexpr int kAPad = round_up(kABytes, 1024);
     static constexpr int kBPad = round_up(kAtoms * kBAtomBytes, 1024);
-    static constexpr int kStageBytes = kAPad + kBPad;
     static constexpr uint32_t kBLayout = kAtomRowBytes == 128 ? 2u : (kAtomRowBytes == 64 ? 4u : 6u);
     static constexpr uint32_t kBSbo = 8 * kAtomRowBytes;
     static_assert(kAtoms == 1 || kBAtomBytes % 1024 == 0, "B atoms must keep the swizzle alignment");
+    static_assert(kJobRows % kWarpRows == 0, "a job must split into whole warp passes");
     static constexpr int kNAlign = BM == 128 ? 16 : 8;
     static constexpr int kChPerWarp = BM / 4;                     // channels of one TMEM lane quarter
-
-    static constexpr int kEntryJBytes = kMaxEntries * 4;           // neighbour rows of the tile's entries
-    static constexpr int kEntryRBytes = kMaxEntries * 2;           // local rows of the tile's entries
-    static constexpr int kCntBytes = 2 * kTileCountStride * 4;     // unit counts, then unit starts
     static constexpr int kOutStageBytes = kFoldWarps * 32 * kChPerWarp * 2;
-    static constexpr int kMetaBytes = kEntryJBytes + kEntryRBytes + kCntBytes + kOutStageBytes + 64 * 8 + 32;
+    static constexpr int kFixedMeta = kMaxJobs * 16 + 2 * kTileCountStride * 4;
 
-    static int stages() {
-        int s = (kMaxSmem - 1024 - kMetaBytes) / kStageBytes;
-        return s > 8 ? 8 : s;
+    __host__ __device__ static int ring_bytes(int sa, int sb) { return sa * kAPad + kGatherWarps * sb * kBPad; }
+    __host__ __device__ static int num_bars(int sa, int sb) { return 2 * sa + 2 * kGatherWarps * sb + 2 * kScratchBufs + 2; }
+    __host__ __device__ static int smem_bytes(int cap, int sa, int sb) {
+        return 1024 + ring_bytes(sa, sb) + kFixedMeta + cap * 4 + round_up(cap * 2, 16) + num_bars(sa, sb) * 8 + 16;
     }
-    static int smem_bytes(int stages) { return 1024 + stages * kStageBytes + kMetaBytes; }
+    static bool fits(int cap, int sa, int sb) {
+        return smem_bytes(cap, sa, sb) <= kMaxSmem && ring_bytes(sa, sb) >= kOutStageBytes;
+    }
+    // Ring depths for a tile entry capacity `cap`: the deepest weight ring that
+    // fits beside one gather slot per warp (one job per offset is the common case,
+    // so most jobs wait on a fresh weight tile), then the room left to gather
+    // slots; {0, 0} if nothing fits.
+    static void depths(int cap, int* sa, int* sb) {
+        *sa = 0;
+        *sb = 0;
+        int a = kMaxASlots;
+        while (a >= 2 && !fits(cap, a, 1)) --a;
+        if (a < 2) return;
+        int b = 1;
+        while (b < kMaxBSlots && fits(cap, a, b + 1)) ++b;
+        *sa = a;
+        *sb = b;
+    }
 };
 
 struct Params {
@@ -110,118 +144,42 @@ struct Params {
     __nv_bfloat16* out;
     int cout;
     unsigned int* err;
-    int stages;
+    int sa;   // weight ring slots
+    int sb;   // gather slots per gather warp
+    int cap;  // entry capacity of the shared-memory lists (largest tile's entries)
 };
 
-// A unit of MMA work: one offset, up to 128 (centre) or 48 (other) columns.
-struct Job {
-    int k;       // offset (13 = centre for kernel size 3; 0 for kernel size 1)
-    int ks;      // index among the 26 non-centre offsets (other offsets)
-    int base;    // flat index of the offset's first entry in the tile metadata
-    int first;   // first row (centre) or first entry of the offset's list (other offsets)
-    int n;       // valid columns
-    int ncols;   // MMA N (n rounded up)
-    bool centre;
-};
-
-// Per-offset hit lists come from the tile metadata built with the map: offset
-// k's entries are the concatenation of its three classes (rows r with r % 3 ==
-// 0, 1, 2, each sorted by row), flat indices ustart[3 ks] .. ustart[3 ks + 3).
-// Enumerates the jobs of a tile in issue order: centre slices, then the other 26
-// offsets, each split into kScratchCols-wide parts.  The order of the 26 offsets
-// is rotated per CTA (`rot`) so that CTAs running at the same time request
-// different weight tiles instead of all reading the same L2 lines.  Every role
-// of a CTA walks the same sequence.
-struct JobIter {
-    const int* ustart;  // unit starts, ustart[kTileUnits] = number of entries
-    int t_eff, kvol, nalign, rot;
-    int ki, k, ks, first, total;  // ki: position among the 26 non-centre offsets
-    __device__ void start() {
-        ki = -1;
-        first = 0;
-    }
-    __device__ void set_offset() {
-        ks = (ki + rot) % (kVol3 - 1);
-        k = ks < kCentre ? ks : ks + 1;
-        total = ustart[3 * ks + 3] - ustart[3 * ks];
-        first = 0;
-    }
-    __device__ bool next(Job& j) {
-        if (ki == -1) {
-            if (first < t_eff) {
-                j.k = kvol == kVol3 ? kCentre : 0;
-                j.ks = 0;
-                j.base = 0;
-                j.first = first;
-                j.n = min(kCentreCols, t_eff - first);
-                j.ncols = round_up(j.n, nalign);
-                j.centre = true;
-                first += kCentreCols;
-                return true;
-            }
-            if (kvol != kVol3) return false;
-            ki = 0;
-            set_offset();
-        }
-        while (ki < kVol3 - 1) {
-            if (first < total) {
-                j.k = k;
-                j.ks = ks;
-                j.base = ustart[3 * ks];
-                j.first = first;
-                j.n = min(kScratchCols, total - first);
-                j.ncols = round_up(j.n, nalign);
-                j.centre = false;
-                first += kScratchCols;
-                return true;
-            }
-            if (++ki < kVol3 - 1) set_offset();
-        }
-        return false;
-    }
-};
-
-// Bounded wait on an mbarrier phase.  `backoff` lets a non-critical waiter sleep
-// between polls so that it does not take issue slots from the MMA issuer.
-template <bool backoff = false>
+// Bounded wait on an mbarrier phase.  By default the thread sleeps inside
+// try_wait; kSpin polls with test_wait instead (lowest wake-up latency, for the
+// single-thread roles on the critical path).
+template <bool kSpin = false>
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                          unsigned int* err) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (kSpin ? mbar_test_wait(bar, parity) : mbar_try_wait_hint(bar, parity, kSuspendHintNs)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 1;; ++i) {
-        if (backoff) __nanosleep(64);
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 63) == 0) {
-            if (*abort_flag) return false;
-            if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
-                *abort_flag = 1;
-                atomicOr(err, kFwdErrTimeout);
-                return false;
-            }
+        if (kSpin ? mbar_test_wait(bar, parity) : mbar_try_wait_hint(bar, parity, kSuspendHintNs)) return true;
+        if (kSpin && (i & 255) != 0) continue;
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+            *abort_flag = 1;
+            atomicOr(err, kFwdErrTimeout);
+            return false;
         }
     }
+}
+
+// Lane 0 waits, the warp learns the outcome.
+__device__ __forceinline__ bool warp_wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                              unsigned int* err) {
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, abort_flag, err) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
 __device__ __forceinline__ void named_barrier(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
-
-// Group wait: one thread of the group polls the mbarrier, the whole group then
-// meets at a hardware named barrier (blocked warps take no issue slots).  The
-// result travels through one of two alternating shared-memory slots.
-struct GroupWait {
-    int barrier_id, nthreads;
-    bool leader;
-    volatile int* slots;  // two ints
-    int phase;
-    __device__ bool operator()(uint32_t bar, uint32_t parity, volatile int* abort_flag, unsigned int* err) {
-        volatile int* slot = slots + (phase & 1);
-        ++phase;
-        if (leader) *slot = wait_bar<true>(bar, parity, abort_flag, err) ? 1 : 0;
-        named_barrier(barrier_id, nthreads);
-        return *slot != 0;
-    }
-};
 
 template <int BM, int KC>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -229,21 +187,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     using L = Layout<BM, KC>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int S = p.stages;
-    uint8_t* stages = smem;
-    int32_t* pj_s = reinterpret_cast<int32_t*>(smem + S * L::kStageBytes);
-    uint16_t* pr_s = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(pj_s) + L::kEntryJBytes);
-    int* cnt = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(pr_s) + L::kEntryRBytes);
+    const int SA = p.sa, SB = p.sb;
+    uint8_t* a_ring = smem;
+    uint8_t* b_ring = smem + SA * L::kAPad;
+    int4* jobs = reinterpret_cast<int4*>(smem + L::ring_bytes(SA, SB));
+    int* cnt = reinterpret_cast<int*>(jobs + kMaxJobs);
     int* ustart = cnt + kTileCountStride;
-    __nv_bfloat16* out_stage = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(cnt) + L::kCntBytes);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(out_stage) + L::kOutStageBytes);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 6);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    volatile int* wait_slots = abort_flag + 1;  // 2 for the gather group, 2 for the fold group
+    int32_t* pj_s = reinterpret_cast<int32_t*>(ustart + kTileCountStride);
+    uint16_t* pr_s = reinterpret_cast<uint16_t*>(pj_s + p.cap);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(pr_s) + round_up(p.cap * 2, 16));
+    int* misc = reinterpret_cast<int*>(bars + L::num_bars(SA, SB));
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
+    volatile int* abort_flag = misc + 1;
+    __nv_bfloat16* out_stage = reinterpret_cast<__nv_bfloat16*>(smem);
 
-    const uint32_t full0 = smem_addr(bars), empty0 = smem_addr(bars + S);
-    const uint32_t sfull0 = smem_addr(bars + 2 * S), sempty0 = smem_addr(bars + 2 * S + 2);
-    const uint32_t accfull = smem_addr(bars + 2 * S + 4), drain = smem_addr(bars + 2 * S + 5);
+    const uint32_t fullA0 = smem_addr(bars), emptyA0 = fullA0 + 8 * SA;
+    const uint32_t fullB0 = emptyA0 + 8 * SA, emptyB0 = fullB0 + 8 * kGatherWarps * SB;
+    const uint32_t sfull0 = emptyB0 + 8 * kGatherWarps * SB, sempty0 = sfull0 + 8 * kScratchBufs;
+    const uint32_t accfull = sempty0 + 8 * kScratchBufs, drain = accfull + 8;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t row0 = (int64_t)blockIdx.x * kTileRows;
@@ -251,13 +212,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int cblk = blockIdx.y;
     const int nchunks = p.cin / KC;
 
-    // ---- set-up: barriers, TMEM, neighbour rows of the tile (cp.async, 16 B)
+    // ---- set-up: barriers, TMEM, the tile's lists (cp.async, 16 B)
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(full0 + 8 * s, 1 + kGatherThreads);  // weight TMA + every gather thread
-            mbar_init(empty0 + 8 * s, 1);
+        for (int s = 0; s < SA; ++s) {
+            mbar_init(fullA0 + 8 * s, 1);
+            mbar_init(emptyA0 + 8 * s, 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int s = 0; s < kGatherWarps * SB; ++s) {
+            mbar_init(fullB0 + 8 * s, 32);  // the 32 lanes of the filling gather warp
+            mbar_init(emptyB0 + 8 * s, 1);
+        }
+        for (int b = 0; b < kScratchBufs; ++b) {
             mbar_init(sfull0 + 8 * b, 1);
             mbar_init(sempty0 + 8 * b, kFoldWarps);
         }
@@ -272,9 +237,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_relinquish();
     }
     if (p.kvol == kVol3) {
-        // The tile's metadata: unit counts (320 B) and entries (local row, neighbour
-        // row); every tile's entries start on a multiple of 8, so all copies are
-        // 16-byte aligned.
+        // Unit counts (320 B) and entries (neighbour row, local row); every tile's
+        // entries start on a multiple of 8, so all copies are 16-byte aligned.
         const int64_t e0 = p.tile_off[blockIdx.x], ne = p.tile_off[blockIdx.x + 1] - e0;
         const uint32_t cnt_dst = smem_addr(cnt), pj_dst = smem_addr(pj_s), pr_dst = smem_addr(pr_s);
         const int32_t* cnt_src = p.tile_counts + (int64_t)blockIdx.x * kTileCountStride;
@@ -288,47 +252,91 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    // ---- flat start of every (offset, class) unit
-    if (p.kvol == kVol3 && warp == 0) {
-        int run = 0;
-        for (int base = 0; base < kTileUnits; base += 32) {
-            const int u = base + lane;
-            const int c = u < kTileUnits ? cnt[u] : 0;
-            int incl = c;
+    // ---- job table (warp 0): centre slices, then every other offset's list in
+    // 48-entry parts.  The order of the 26 offsets is rotated per CTA so that
+    // CTAs running at the same time request different weight tiles.
+    if (warp == 0) {
+        const int kc = p.kvol == kVol3 ? kCentre : 0;
+        const int ncj = (t_eff + kJobRows - 1) / kJobRows;
+        for (int j = lane; j < ncj; j += 32) {
+            const int n = min(kJobRows, t_eff - j * kJobRows);
+            jobs[j] = make_int4(kc | (1 << 16), j * kJobRows, n, round_up(n, L::kNAlign));
+        }
+        int njobs = ncj;
+        if (p.kvol == kVol3) {
+            int run = 0;  // flat start of every (offset, class) unit
+            for (int base = 0; base < kTileUnits; base += 32) {
+                const int u = base + lane;
+                const int c = u < kTileUnits ? cnt[u] : 0;
+                int incl = c;
+#pragma unroll
+                for (int d = 1; d < 32; d <<= 1) {
+                    const int v = __shfl_up_sync(0xffffffffu, incl, d);
+                    if (lane >= d) incl += v;
+                }
+                if (u < kTileUnits) ustart[u] = run + incl - c;
+                run += __shfl_sync(0xffffffffu, incl, 31);
+            }
+            if (lane == 0) ustart[kTileUnits] = run;
+            __syncwarp();
+            const int rot = (int)((blockIdx.x * 11u + blockIdx.y * 5u) % (kVol3 - 1));
+            int ks = 0, e0 = 0, tot = 0, nj = 0;
+            if (lane < kVol3 - 1) {
+                ks = (lane + rot) % (kVol3 - 1);
+                e0 = ustart[3 * ks];
+                tot = ustart[3 * ks + 3] - e0;
+                nj = (tot + kJobRows - 1) / kJobRows;
+            }
+            int incl = nj;
 #pragma unroll
             for (int d = 1; d < 32; d <<= 1) {
                 const int v = __shfl_up_sync(0xffffffffu, incl, d);
                 if (lane >= d) incl += v;
             }
-            if (u < kTileUnits) ustart[u] = run + incl - c;
-            run += __shfl_sync(0xffffffffu, incl, 31);
+            const int start = ncj + incl - nj;
+            const int k = ks < kCentre ? ks : ks + 1;
+            for (int q = 0; q < nj; ++q) {
+                const int n = min(kJobRows, tot - q * kJobRows);
+                jobs[start + q] = make_int4(k | (ks << 8), e0 + q * kJobRows, n, round_up(n, L::kNAlign));
+            }
+            njobs = ncj + __shfl_sync(0xffffffffu, incl, 31);
         }
-        if (lane == 0) ustart[kTileUnits] = run;
+        __syncwarp();
+        // first gather slot and phase of every job: the job is the (j / 4)-th of
+        // gather warp j % 4, whose ring has advanced by nchunks per earlier job
+        for (int j = lane; j < njobs; j += 32) {
+            const int u0 = (j / kGatherWarps) * nchunks;
+            jobs[j].x |= ((u0 % SB) << 17) | (((u0 / SB) & 1) << 20);
+        }
+        if (lane == 0) misc[2] = njobs;
     }
     __syncthreads();
-
-    JobIter it_jobs{ustart, t_eff, p.kvol, L::kNAlign, (int)((blockIdx.x * 11u + blockIdx.y * 5u) % (kVol3 - 1)),
-                    0, 0, 0, 0, 0};
-    Job job;
+    const int njobs = misc[2];
     bool aborted = false;
 
     if (warp == kWarpTma) {
         // ------------------------------------------------ weights via TMA
         if (lane == 0) {
-            int it = 0;
-            it_jobs.start();
-            while (!aborted && it_jobs.next(job)) {
-                for (int c = 0; c < nchunks; ++c, ++it) {
-                    const int s = it % S;
-                    if (!wait_bar<true>(empty0 + 8 * s, ((uint32_t)(it / S) & 1u) ^ 1u, abort_flag, p.err)) {
+            int s = 0, prev_k = -1;
+            uint32_t ph = 0;
+            for (int j = 0; j < njobs && !aborted; ++j) {
+                const int k = job_k(jobs[j]);
+                if (nchunks == 1 && k == prev_k) continue;  // same offset: the loaded tile serves
+                prev_k = k;
+                for (int c = 0; c < nchunks; ++c) {
+                    if (!wait_bar(emptyA0 + 8 * s, ph ^ 1u, abort_flag, p.err)) {
                         aborted = true;
                         break;
                     }
-                    const uint32_t a_dst = smem_addr(stages + s * L::kStageBytes);
-                    mbar_arrive_expect_tx(full0 + 8 * s, L::kABytes);
-                    const int y = job.k * p.cin + c * KC;
+                    const uint32_t a_dst = smem_addr(a_ring + s * L::kAPad);
+                    mbar_arrive_expect_tx(fullA0 + 8 * s, L::kABytes);
+                    const int y = k * p.cin + c * KC;
                     for (int box = 0; box < BM / 64; ++box)
-                        tma_load_2d(a_dst + box * KC * 128, &wmap, cblk * BM + box * 64, y, full0 + 8 * s);
+                        tma_load_2d(a_dst + box * KC * 128, &wmap, cblk * BM + box * 64, y, fullA0 + 8 * s);
+                    if (++s == SA) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
             }
             if (aborted) __nanosleep(200000);  // let loads in flight land before the CTA exits
@@ -336,27 +344,56 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == kWarpMma) {
         // ------------------------------------------------ tcgen05.mma issuer
         if (lane == 0) {
-            int it = 0, sj = 0;
-            it_jobs.start();
-            while (!aborted && it_jobs.next(job)) {
-                const uint32_t d =
-                    tmem + (job.centre ? (uint32_t)job.first : kScratchCol0 + (uint32_t)(sj & 1) * kScratchCols);
-                if (!job.centre) {
-                    if (!wait_bar(sempty0 + 8 * (sj & 1), ((uint32_t)(sj >> 1) & 1u) ^ 1u, abort_flag, p.err)) {
+            int as = SA - 1, prev_k = -1;  // weight slot in use and its phase
+            uint32_t aph = 1u;
+            int sb_ = kScratchBufs - 1;  // scratch buffer of the last offset job and its phase
+            uint32_t sph = 1u;
+            int4 jb = njobs > 0 ? jobs[0] : make_int4(0, 0, 0, 0);
+            for (int j = 0; j < njobs && !aborted; ++j) {
+                const int4 jn = j + 1 < njobs ? jobs[j + 1] : make_int4(-1, 0, 0, 0);  // prefetch
+                const int k = job_k(jb);
+                const bool centre = job_centre(jb);
+                const bool new_k = k != prev_k;
+                prev_k = k;
+                const bool last_of_k = j + 1 == njobs || job_k(jn) != k;
+                uint32_t d = tmem + (uint32_t)jb.y;
+                if (!centre) {
+                    if (++sb_ == kScratchBufs) {
+                        sb_ = 0;
+                        sph ^= 1u;
+                    }
+                    d = tmem + kScratchCol0 + (uint32_t)sb_ * kJobRows;
+                    if (!wait_bar(sempty0 + 8 * sb_, sph ^ 1u, abort_flag, p.err)) {
                         aborted = true;
                         break;
                     }
+                    tc_fence_after();
                 }
-                const uint32_t idesc = idesc_bf16(BM, (uint32_t)job.ncols);
-                for (int c = 0; c < nchunks; ++c, ++it) {
-                    const int s = it % S;
-                    const uint32_t ph = (uint32_t)(it / S) & 1u;
-                    if (!wait_bar(full0 + 8 * s, ph, abort_flag, p.err)) {
+                const uint32_t idesc = idesc_bf16(BM, (uint32_t)jb.w);
+                const int gw = j & (kGatherWarps - 1);
+                int bs = job_bslot(jb);
+                uint32_t bph = job_bphase(jb);
+                for (int c = 0; c < nchunks; ++c) {
+                    if (nchunks > 1 || (c == 0 && new_k)) {
+                        if (++as == SA) {
+                            as = 0;
+                            aph ^= 1u;
+                        }
+                        if (!wait_bar(fullA0 + 8 * as, aph, abort_flag, p.err)) {
+                            aborted = true;
+                            break;
+                        }
+                    }
+                    const int bslot = gw * SB + bs;
+                    if (!wait_bar(fullB0 + 8 * bslot, bph, abort_flag, p.err)) {
                         aborted = true;
                         break;
                     }
-                    const uint32_t a_base = smem_addr(stages + s * L::kStageBytes);
-                    const uint32_t b_base = a_base + L::kAPad;
+                    // the B tile was written by cp.async (generic proxy); the MMA reads it
+                    // through the async proxy
+                    fence_proxy_async_smem();
+                    const uint32_t a_base = smem_addr(a_ring + as * L::kAPad);
+                    const uint32_t b_base = smem_addr(b_ring + bslot * L::kBPad);
 #pragma unroll
                     for (int kk = 0; kk < KC / 16; ++kk) {
                         const uint64_t adesc = smem_desc(a_base + kk * 2048, KC * 128, 1024, 2);
@@ -366,13 +403,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                                       L::kBSbo, L::kBLayout);
                         mma_bf16(d, adesc, bdesc, idesc, (c > 0 || kk > 0) ? 1u : 0u);
                     }
-                    mma_commit(empty0 + 8 * s);
+                    mma_commit(emptyB0 + 8 * bslot);
+                    if (nchunks > 1 || last_of_k) mma_commit(emptyA0 + 8 * as);
+                    if (++bs == SB) {
+                        bs = 0;
+                        bph ^= 1u;
+                    }
                 }
                 if (aborted) break;
-                if (!job.centre) {
-                    mma_commit(sfull0 + 8 * (sj & 1));
-                    ++sj;
-                }
+                if (!centre) mma_commit(sfull0 + 8 * sb_);
+                jb = jn;
             }
             if (!aborted) {
                 mma_commit(accfull);
@@ -385,48 +425,51 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp < kWarpFold0) {
         // ------------------------------------------------ gather producers
-        // The four warps fill every stage together.  Per job: resolve this
-        // thread's source rows once (independent shared-memory lookups), then
-        // issue the 16-byte copies of every input-channel chunk.  Each thread
-        // arrives on the stage barrier when its own copies land
-        // (cp.async.mbarrier.arrive.noinc), so no producer ever waits for data.
-        constexpr int kMaxPass = (kJobRows + L::kRowsPerPass - 1) / L::kRowsPerPass;
-        const int g = threadIdx.x - kWarpGather0 * 32;
-        GroupWait gwait{3, kGatherThreads, g == 0, wait_slots, 0};
-        const int q = g % L::kThreadsPerRow;
-        const int prow = g / L::kThreadsPerRow;
+        // Lane l copies 16-byte chunk l % kThreadsPerRow of rows
+        // l / kThreadsPerRow + kWarpRows * pass; the job's source rows are looked
+        // up once and serve every channel chunk.  Each lane arrives on the slot's
+        // barrier when its own copies land (cp.async.mbarrier.arrive.noinc), so no
+        // producer ever waits for data.
+        const int gw = warp - kWarpGather0;
+        const int q = lane % L::kThreadsPerRow;
+        const int prow = lane / L::kThreadsPerRow;
         const int atom = q / L::kChunksPerAtom, qa = q % L::kChunksPerAtom;
-        int it = 0;
-        it_jobs.start();
-        while (!aborted && it_jobs.next(job)) {
-            int64_t src_row[kMaxPass];
-            uint32_t dst_off[kMaxPass];
+        int s = 0;
+        uint32_t ph = 0;
+        for (int j = gw; j < njobs && !aborted; j += kGatherWarps) {
+            const int4 jb = jobs[j];
+            const bool centre = job_centre(jb);
+            const int n = jb.z, ncols = jb.w;
+            int src[L::kPasses];
 #pragma unroll
-            for (int ps = 0; ps < kMaxPass; ++ps) {
-                const int pr = prow + ps * L::kRowsPerPass;
-                src_row[ps] = -1;
-                if (pr < job.n) src_row[ps] = job.centre ? row0 + job.first + pr : (int64_t)pj_s[job.base + job.first + pr];
-                const uint32_t lin = (uint32_t)(pr * L::kAtomRowBytes + qa * 16);
-                dst_off[ps] = (uint32_t)(atom * L::kBAtomBytes) + (lin ^ (((lin >> 7) & L::kSwizzleMask) << 4));
+            for (int ps = 0; ps < L::kPasses; ++ps) {
+                const int pr = prow + ps * L::kWarpRows;
+                src[ps] = -1;
+                if (pr < n) src[ps] = centre ? (int)row0 + jb.y + pr : pj_s[jb.y + pr];
             }
-            for (int c = 0; c < nchunks; ++c, ++it) {
-                const int s = it % S;
-                const uint32_t ph = (uint32_t)(it / S) & 1u;
-                if (!gwait(empty0 + 8 * s, ph ^ 1u, abort_flag, p.err)) {
+            for (int c = 0; c < nchunks; ++c) {
+                const int slot = gw * SB + s;
+                if (!warp_wait_bar(emptyB0 + 8 * slot, ph ^ 1u, abort_flag, p.err)) {
                     aborted = true;
                     break;
                 }
-                const uint32_t b_base = smem_addr(stages + s * L::kStageBytes) + L::kAPad;
+                const uint32_t b_base = smem_addr(b_ring + slot * L::kBPad) + (uint32_t)(atom * L::kBAtomBytes);
+                const __nv_bfloat16* xc = p.x + c * KC + q * 8;
 #pragma unroll
-                for (int ps = 0; ps < kMaxPass; ++ps) {
-                    const int pr = prow + ps * L::kRowsPerPass;
-                    if (pr < job.ncols) {
-                        const bool hit = src_row[ps] >= 0;
-                        cp_async_16(b_base + dst_off[ps], p.x + (hit ? src_row[ps] : 0) * p.cin + c * KC + q * 8,
-                                    hit ? 16u : 0u);
+                for (int ps = 0; ps < L::kPasses; ++ps) {
+                    const int pr = prow + ps * L::kWarpRows;
+                    if (pr < ncols) {
+                        const uint32_t lin = (uint32_t)(pr * L::kAtomRowBytes + qa * 16);
+                        const bool hit = src[ps] >= 0;
+                        cp_async_16(b_base + (lin ^ (((lin >> 7) & L::kSwizzleMask) << 4)),
+                                    xc + (int64_t)(hit ? src[ps] : 0) * p.cin, hit ? 16u : 0u);
                     }
                 }
-                cp_async_mbar_arrive_noinc(full0 + 8 * s);
+                cp_async_mbar_arrive_noinc(fullB0 + 8 * slot);
+                if (++s == SB) {
+                    s = 0;
+                    ph ^= 1u;
+                }
             }
         }
         cp_async_wait_all();
@@ -437,37 +480,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         // one warp per lane quarter.
         const int quarter = warp & 3;
         const int sub = (warp - kWarpFold0) >> 2;
-        GroupWait fwait{2, 32 * kFoldWarps, threadIdx.x == kWarpFold0 * 32, wait_slots + 2, 0};
         const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
-        int sj = 0;
-        it_jobs.start();
-        while (!aborted && it_jobs.next(job)) {
-            if (job.centre) continue;
-            const int b = sj & 1;
-            if (!fwait(sfull0 + 8 * b, (uint32_t)(sj >> 1) & 1u, abort_flag, p.err)) {
+        int b = kScratchBufs - 1;  // scratch buffer of the current offset job and its phase
+        uint32_t sph = 1u;
+        for (int j = 0; j < njobs; ++j) {
+            const int4 jb = jobs[j];
+            if (job_centre(jb)) continue;
+            if (++b == kScratchBufs) {
+                b = 0;
+                sph ^= 1u;
+            }
+            if (!warp_wait_bar(sfull0 + 8 * b, sph, abort_flag, p.err)) {
                 aborted = true;
                 break;
             }
-            const uint32_t scr = tmem + lane_base + kScratchCol0 + (uint32_t)b * kScratchCols;
-            // this warp's class of the job's offset: flat entries [cls_lo, cls_hi)
-            const int cls_lo = ustart[3 * job.ks + sub] - job.base, cls_hi = ustart[3 * job.ks + sub + 1] - job.base;
-            const int lo = max(job.first, cls_lo);
-            const int hi = min(job.first + job.n, cls_hi);
-            const uint16_t* lst = pr_s + job.base;
+            tc_fence_after();
+            const uint32_t scr = tmem + lane_base + kScratchCol0 + (uint32_t)b * kJobRows;
+            // this warp's class of the job's offset: flat entries [lo, hi)
+            const int ks = job_ks(jb), first = jb.y;
+            const int lo = max(first, ustart[3 * ks + sub]);
+            const int hi = min(first + jb.z, ustart[3 * ks + sub + 1]);
             // 1) read this warp's scratch columns with wide loads and hand the
             //    buffer back to the MMA issuer at once;
-            float v[kScratchCols];
-            const int ng = (hi - lo + kFoldGroup - 1) / kFoldGroup;  // <= 3
-            if (ng > 0) tmem_ld_x16(scr + (uint32_t)(lo - job.first), v);
-            if (ng > 1) tmem_ld_x16(scr + (uint32_t)(lo - job.first + kFoldGroup), v + kFoldGroup);
-            if (ng > 2) tmem_ld_x16(scr + (uint32_t)(lo - job.first + 2 * kFoldGroup), v + 2 * kFoldGroup);
+            float v[kJobRows];
+            const int ng = hi > lo ? (hi - lo + kFoldGroup - 1) / kFoldGroup : 0;  // <= 3
+            if (ng > 0) tmem_ld_x16(scr + (uint32_t)(lo - first), v);
+            if (ng > 1) tmem_ld_x16(scr + (uint32_t)(lo - first + kFoldGroup), v + kFoldGroup);
+            if (ng > 2) tmem_ld_x16(scr + (uint32_t)(lo - first + 2 * kFoldGroup), v + 2 * kFoldGroup);
             tmem_wait_ld();  // the scratch values are in registers
+            tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(sempty0 + 8 * b);
             // 2) then add them into the accumulator columns of their rows.
             if (ng > 0) tmem_wait_st();  // this warp's stores of the previous job have landed
 #pragma unroll
-            for (int gi = 0; gi < kScratchCols / kFoldGroup; ++gi) {
+            for (int gi = 0; gi < kJobRows / kFoldGroup; ++gi) {
                 if (gi < ng) {
                     const int g0 = lo + gi * kFoldGroup;
                     float a[kFoldGroup];
@@ -475,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int i = 0; i < kFoldGroup; ++i) {
                         const int e = g0 + i;
-                        const uint32_t r = lst[min(e, hi - 1)];
+                        const uint32_t r = pr_s[min(e, hi - 1)];
                         col[i] = tmem + lane_base + (e < hi ? r : kDummyCol0 + (uint32_t)i);
                         tmem_ld_x1(col[i], a[i]);
                     }
@@ -484,12 +531,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int i = 0; i < kFoldGroup; ++i) tmem_st_x1(col[i], a[i] + v[gi * kFoldGroup + i]);
                 }
             }
-            ++sj;
         }
         tmem_wait_st();
         tc_fence_before();
         named_barrier(1, 32 * kFoldWarps);  // every fold store has landed before any epilogue read
-        if (!aborted && fwait(accfull, 0, abort_flag, p.err)) {
+        if (!aborted && warp_wait_bar(accfull, 0, abort_flag, p.err)) {
             tc_fence_after();
             const bool lane_ok = lane < L::kChPerWarp;
             const int ch_base = cblk * BM + quarter * L::kChPerWarp;
@@ -557,6 +603,10 @@ spconv_status_t launch(const MapData& m, const void* x, int cin, const void* w, 
         return SPCONV_ERR_CUDA;
     }
     const int kvol = m.kernel_size == 3 ? kVol3 : 1;
+    const int cap = kvol == kVol3 ? (int)m.tile_max_entries : 0;
+    int sa = 0, sb = 0;
+    L::depths(cap, &sa, &sb);
+    if (sa < 2 || sb < 1) return SPCONV_ERR_UNSUPPORTED;
     // Weights [kvol, cin, cout] viewed as 2-D [kvol*cin rows, cout columns]; a box
     // is 64 output channels (128 B, 128-byte swizzle) by KC input channels.
     CUtensorMap map;
@@ -571,12 +621,11 @@ spconv_status_t launch(const MapData& m, const void* x, int cin, const void* w, 
         *ce = cudaErrorInvalidValue;
         return SPCONV_ERR_CUDA;
     }
-    const int stages = L::stages();
-    const int smem = L::smem_bytes(stages);
+    const int smem = L::smem_bytes(cap, sa, sb);
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [&] {
-        attr_err = cudaFuncSetAttribute(k_subm_tc<BM, KC>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        attr_err = cudaFuncSetAttribute(k_subm_tc<BM, KC>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
     });
     if (attr_err != cudaSuccess) {
         *ce = attr_err;
@@ -595,7 +644,9 @@ spconv_status_t launch(const MapData& m, const void* x, int cin, const void* w, 
     p.out = static_cast<__nv_bfloat16*>(out);
     p.cout = cout;
     p.err = m.fwd_err;
-    p.stages = stages;
+    p.sa = sa;
+    p.sb = sb;
+    p.cap = cap;
     dim3 grid((unsigned)((m.n + kTileRows - 1) / kTileRows), (unsigned)((cout + BM - 1) / BM));
     k_subm_tc<BM, KC><<<grid, kThreads, smem, stream>>>(map, p);
     *ce = cudaGetLastError();

@@ -174,23 +174,31 @@ __global__ void k_tile_count(const int32_t* __restrict__ nbr, int64_t n, int32_t
 }
 
 // Exclusive scan of the per-tile totals (in place, one CTA): off[t] = sum of
-// totals before t; off[ntiles] = grand total.
+// totals before t; off[ntiles] = grand total; off[ntiles + 1] = largest total
+// of one tile (the forward kernel sizes its shared-memory entry lists by it).
 __global__ void k_tile_scan(int64_t* __restrict__ off, int64_t ntiles) {
     __shared__ int64_t part[1024];
+    __shared__ int64_t pmax[1024];
     const int64_t per = (ntiles + blockDim.x - 1) / blockDim.x;
     const int64_t lo = threadIdx.x * per, hi = min(ntiles, lo + per);
-    int64_t sum = 0;
-    for (int64_t i = lo; i < hi; ++i) sum += off[i];
+    int64_t sum = 0, mx = 0;
+    for (int64_t i = lo; i < hi; ++i) {
+        sum += off[i];
+        mx = max(mx, off[i]);
+    }
     part[threadIdx.x] = sum;
+    pmax[threadIdx.x] = mx;
     __syncthreads();
     if (threadIdx.x == 0) {
-        int64_t run = 0;
+        int64_t run = 0, m = 0;
         for (int i = 0; i < (int)blockDim.x; ++i) {
             const int64_t v = part[i];
             part[i] = run;
             run += v;
+            m = max(m, pmax[i]);
         }
         off[ntiles] = run;
+        off[ntiles + 1] = m;
     }
     __syncthreads();
     int64_t run = part[threadIdx.x];
@@ -248,7 +256,7 @@ __global__ void k_tile_fill(const int32_t* __restrict__ nbr, int64_t n, const in
 cudaError_t launch_tile_count(const int32_t* nbr, int64_t n, int32_t* tile_counts, int64_t* tile_off,
                               cudaStream_t stream) {
     const int64_t nt = num_tiles(n);
-    if (nt == 0) return cudaMemsetAsync(tile_off, 0, sizeof(int64_t), stream);
+    if (nt == 0) return cudaMemsetAsync(tile_off, 0, 2 * sizeof(int64_t), stream);
     k_tile_count<<<(unsigned)nt, kMetaThreads, 0, stream>>>(nbr, n, tile_counts, tile_off);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;

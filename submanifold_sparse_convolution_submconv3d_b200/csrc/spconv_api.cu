@@ -85,18 +85,20 @@ spconv_status_t spconv_build_map(const int32_t* coords, int64_t n, const int32_t
     const int64_t ntiles = spconv::num_tiles(n);
     const bool tiles = kernel_size == 3 && n > 0;
     if (e == cudaSuccess && tiles) e = cudaMalloc(&m->d.tile_counts, (size_t)ntiles * spconv::kTileCountStride * 4);
-    if (e == cudaSuccess && tiles) e = cudaMalloc(&m->d.tile_off, (size_t)(ntiles + 1) * sizeof(int64_t));
+    if (e == cudaSuccess && tiles) e = cudaMalloc(&m->d.tile_off, (size_t)(ntiles + 2) * sizeof(int64_t));
     if (e == cudaSuccess)
         e = spconv::launch_build_map(coords, n, extent, kernel_size, table, slots, m->d.nbr, flags, stream);
     if (e == cudaSuccess && tiles) e = spconv::launch_tile_count(m->d.nbr, n, m->d.tile_counts, m->d.tile_off, stream);
-    int64_t total_entries = 0;
+    int64_t entry_stats[2] = {0, 0};  // grand total, largest tile
     if (e == cudaSuccess && tiles)
-        e = cudaMemcpyAsync(&total_entries, m->d.tile_off + ntiles, sizeof(int64_t), cudaMemcpyDeviceToHost, stream);
+        e = cudaMemcpyAsync(entry_stats, m->d.tile_off + ntiles, sizeof(entry_stats), cudaMemcpyDeviceToHost, stream);
+    const int64_t total_entries = entry_stats[0];
     if (e == cudaSuccess) e = cudaMemcpyAsync(&host_flags, flags, sizeof(host_flags), cudaMemcpyDeviceToHost, stream);
     if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
     // Second phase (only if the map is valid): entry arrays of the tile metadata.
     if (e == cudaSuccess && tiles && host_flags.err == 0) {
         m->d.tile_entries = total_entries;
+        m->d.tile_max_entries = entry_stats[1];
         const size_t ne = total_entries > 0 ? (size_t)total_entries : 1;
         e = cudaMalloc(&m->d.pair_r, ne * sizeof(uint16_t));
         if (e == cudaSuccess) e = cudaMalloc(&m->d.pair_j, ne * sizeof(int32_t));

@@ -113,7 +113,7 @@ def test_dense_block_and_isolated_voxels(sp):
 
 
 def test_single_voxel_and_single_tile_edge(sp):
-    for n in (1, 383, 384, 385):
+    for n in (1, 351, 352, 353, 383, 384, 385, 705):  # around the 384-row tile and other sizes
         coords, ext, x, w, b = _case(6 + n, 12, n, 64, 64)
         out = _run(sp, coords, ext, x, w, b, "bf16", algo=sp.ALGO_TCGEN05)
         assert_close(out, _ref(coords, ext, x, w, b), "bf16")
