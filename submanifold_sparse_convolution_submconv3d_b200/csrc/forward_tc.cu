@@ -11,23 +11,26 @@
 // output channels.  Tensor memory (TMEM, 128 lanes x 512 fp32 columns) holds
 //   * the accumulator: lane = output channel, column = output row of the tile;
 //   * two scratch buffers of kJobRows columns and 16 dummy columns.
-// Work is cut into jobs of at most kJobRows columns, listed once per tile in
-// shared memory: first the centre offset (every row is its own neighbour) in
-// 48-row slices that go straight into the accumulator, then for every other
-// offset the compacted list of tile rows that have a neighbour there.  A job's
-// neighbour feature rows are gathered (cp.async, 16 B, zero-filled padding) into
-// a swizzled shared-memory tile and multiplied into a scratch buffer; fold warps
-// then add each scratch column into the accumulator column of its row
+// Work is cut into jobs listed once per tile in shared memory.  First the centre
+// offset (every row is its own neighbour): its feature rows are contiguous, so
+// they arrive by a tiled TMA load, BM rows per job, and the products go straight
+// into the accumulator; with kernel size 1 this is the whole layer, a plain
+// TMA-fed tensor-core GEMM.  Then, for every other offset, the compacted list of
+// tile rows that have a neighbour there, in parts of at most kJobRows entries:
+// their neighbour feature rows are gathered (cp.async, 16 B, zero-filled padding)
+// into a swizzled shared-memory tile and multiplied into a scratch buffer, and
+// fold warps add each scratch column into the accumulator column of its row
 // (tcgen05.ld / tcgen05.st, no atomics).  W_k arrives by TMA once per offset
-// (once per job and channel chunk when Cin spans several chunks).  At the end
-// each output row is written exactly once, with bias, rounded to bf16.
+// (once per job and channel chunk when Cin spans several chunks, and once per
+// centre job).  At the end each output row is written exactly once, with bias,
+// rounded to bf16.
 //
 // Warp roles (576 threads):
-//   warp 0      TMA producer of weight tiles (A operand), a ring of 2-6 slots
 //   warp 1      TMEM allocator and tcgen05.mma issuer
-//   warps 2-5   gather producers (B operand): warp w fills the jobs j with
-//               j % 4 == w into its own ring of slots, in order, so each ring is
-//               filled and drained strictly in sequence
+//   warp 5      TMA producer of weight tiles (A operand), a ring of 2-6 slots
+//   warps 0, 2-4  gather producers (B operand): gather warp g fills the jobs j
+//               with j % 4 == g into its own ring of slots, in order, so each
+//               ring is filled and drained strictly in sequence
 //   warps 6-17  scratch -> accumulator fold, then the epilogue: three warps per
 //               TMEM lane quarter, each owning the tile rows of one residue mod 3,
 //               so no accumulator column is touched by two warps of a quarter.
@@ -55,7 +58,11 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kScratchCol0 = kTileRows;             // scratch buffer b at column 384 + 48 b
 constexpr uint32_t kDummyCol0 = kScratchCol0 + kScratchBufs * kJobRows;  // 480..495: fold padding targets
 static_assert(kDummyCol0 + 16 <= kTmemCols, "accumulator, scratch buffers and dummy columns must fit TMEM");
-constexpr int kWarpTma = 0, kWarpMma = 1, kWarpGather0 = 2, kWarpFold0 = 6;
+// Warp w runs on sub-partition w % 4, and a fold warp must sit on the
+// sub-partition of its TMEM lane quarter.  The MMA issuer's sub-partition (1)
+// therefore hosts, besides three fold warps, only the light weight producer; the
+// four gather warps (0, 2, 3, 4) go to the others.
+constexpr int kWarpMma = 1, kWarpTma = 5, kWarpFold0 = 6;
 constexpr int kGatherWarps = 4, kFoldWarps = 12;
 constexpr int kThreads = 32 * (kWarpFold0 + kFoldWarps);  // 576
 constexpr int kFoldGroup = 16;
@@ -183,7 +190,7 @@ __device__ __forceinline__ void named_barrier(int id, int nthreads) {
 
 template <int BM, int KC>
 __global__ void __launch_bounds__(kThreads, 1)
-    k_subm_tc(const __grid_constant__ CUtensorMap wmap, const Params p) {
+    k_subm_tc(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap, const Params p) {
     using L = Layout<BM, KC>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -231,6 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tensormap(&wmap);
+        prefetch_tensormap(&xmap);
     }
     if (warp == kWarpMma) {
         tmem_alloc(smem_addr(tmem_slot), kTmemCols);
@@ -252,15 +260,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    // ---- job table (warp 0): centre slices, then every other offset's list in
-    // 48-entry parts.  The order of the 26 offsets is rotated per CTA so that
-    // CTAs running at the same time request different weight tiles.
+    // ---- job table (warp 0): centre slices of BM rows, then every other
+    // offset's list in 48-entry parts.  The order of the 26 offsets is rotated per
+    // CTA so that CTAs running at the same time request different weight tiles.
     if (warp == 0) {
         const int kc = p.kvol == kVol3 ? kCentre : 0;
-        const int ncj = (t_eff + kJobRows - 1) / kJobRows;
+        const int ncj = (t_eff + BM - 1) / BM;
         for (int j = lane; j < ncj; j += 32) {
-            const int n = min(kJobRows, t_eff - j * kJobRows);
-            jobs[j] = make_int4(kc | (1 << 16), j * kJobRows, n, round_up(n, L::kNAlign));
+            const int n = min(BM, t_eff - j * BM);
+            jobs[j] = make_int4(kc | (1 << 16), j * BM, n, round_up(n, L::kNAlign));
         }
         int njobs = ncj;
         if (p.kvol == kVol3) {
@@ -302,40 +310,59 @@ __global__ void __launch_bounds__(kThreads, 1)
             njobs = ncj + __shfl_sync(0xffffffffu, incl, 31);
         }
         __syncwarp();
-        // first gather slot and phase of every job: the job is the (j / 4)-th of
-        // gather warp j % 4, whose ring has advanced by nchunks per earlier job
-        for (int j = lane; j < njobs; j += 32) {
-            const int u0 = (j / kGatherWarps) * nchunks;
+        // first gather slot and phase of every offset job: job ncj + q is the
+        // (q / 4)-th of gather warp q % 4, whose ring has advanced by nchunks per
+        // earlier job
+        for (int j = ncj + lane; j < njobs; j += 32) {
+            const int u0 = ((j - ncj) / kGatherWarps) * nchunks;
             jobs[j].x |= ((u0 % SB) << 17) | (((u0 / SB) & 1) << 20);
         }
-        if (lane == 0) misc[2] = njobs;
+        if (lane == 0) {
+            misc[2] = njobs;
+            misc[3] = ncj;
+        }
     }
     __syncthreads();
-    const int njobs = misc[2];
+    const int njobs = misc[2], ncj = misc[3];
     bool aborted = false;
 
     if (warp == kWarpTma) {
-        // ------------------------------------------------ weights via TMA
+        // ------------------------------------------------ weights (and centre rows) via TMA
+        // Ring uses, in the issuer's order: per centre job and channel chunk the
+        // centre weights then the job's BM feature rows; per offset (per job and
+        // chunk when Cin spans several chunks) the offset's weights.
         if (lane == 0) {
             int s = 0, prev_k = -1;
             uint32_t ph = 0;
             for (int j = 0; j < njobs && !aborted; ++j) {
-                const int k = job_k(jobs[j]);
-                if (nchunks == 1 && k == prev_k) continue;  // same offset: the loaded tile serves
+                const int4 jb = jobs[j];
+                const int k = job_k(jb);
+                const bool centre = job_centre(jb);
+                if (!centre && nchunks == 1 && k == prev_k) continue;  // same offset: the loaded tile serves
                 prev_k = k;
-                for (int c = 0; c < nchunks; ++c) {
-                    if (!wait_bar(emptyA0 + 8 * s, ph ^ 1u, abort_flag, p.err)) {
-                        aborted = true;
-                        break;
-                    }
-                    const uint32_t a_dst = smem_addr(a_ring + s * L::kAPad);
-                    mbar_arrive_expect_tx(fullA0 + 8 * s, L::kABytes);
-                    const int y = k * p.cin + c * KC;
-                    for (int box = 0; box < BM / 64; ++box)
-                        tma_load_2d(a_dst + box * KC * 128, &wmap, cblk * BM + box * 64, y, fullA0 + 8 * s);
-                    if (++s == SA) {
-                        s = 0;
-                        ph ^= 1u;
+                for (int c = 0; c < nchunks && !aborted; ++c) {
+                    for (int part = 0; part < (centre ? 2 : 1); ++part) {
+                        if (!wait_bar(emptyA0 + 8 * s, ph ^ 1u, abort_flag, p.err)) {
+                            aborted = true;
+                            break;
+                        }
+                        const uint32_t dst = smem_addr(a_ring + s * L::kAPad);
+                        mbar_arrive_expect_tx(fullA0 + 8 * s, L::kABytes);
+                        if (part == 0) {
+                            const int y = k * p.cin + c * KC;
+                            for (int box = 0; box < BM / 64; ++box)
+                                tma_load_2d(dst + box * KC * 128, &wmap, cblk * BM + box * 64, y, fullA0 + 8 * s);
+                        } else {
+                            // BM feature rows [row0 + first, +BM) x KC channels, K-major in
+                            // swizzle atoms (rows past the last voxel read as zeros)
+                            for (int a = 0; a < L::kAtoms; ++a)
+                                tma_load_2d(dst + a * BM * L::kAtomRowBytes, &xmap, c * KC + a * L::kAtomElems,
+                                            (int)row0 + jb.y, fullA0 + 8 * s);
+                        }
+                        if (++s == SA) {
+                            s = 0;
+                            ph ^= 1u;
+                        }
                     }
                 }
             }
@@ -370,7 +397,41 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after();
                 }
                 const uint32_t idesc = idesc_bf16(BM, (uint32_t)jb.w);
-                const int gw = j & (kGatherWarps - 1);
+                if (centre) {
+                    // weights and feature rows both come through the TMA ring
+                    for (int c = 0; c < nchunks; ++c) {
+                        int ws = 0;
+                        for (int part = 0; part < 2; ++part) {
+                            if (++as == SA) {
+                                as = 0;
+                                aph ^= 1u;
+                            }
+                            if (part == 0) ws = as;
+                            if (!wait_bar(fullA0 + 8 * as, aph, abort_flag, p.err)) {
+                                aborted = true;
+                                break;
+                            }
+                        }
+                        if (aborted) break;
+                        const uint32_t a_base = smem_addr(a_ring + ws * L::kAPad);
+                        const uint32_t x_base = smem_addr(a_ring + as * L::kAPad);
+#pragma unroll
+                        for (int kk = 0; kk < KC / 16; ++kk) {
+                            const uint64_t adesc = smem_desc(a_base + kk * 2048, KC * 128, 1024, 2);
+                            constexpr int kStepsPerAtom = L::kAtomElems / 16;
+                            const uint64_t bdesc = smem_desc(
+                                x_base + (kk / kStepsPerAtom) * (BM * L::kAtomRowBytes) + (kk % kStepsPerAtom) * 32, 16,
+                                L::kBSbo, L::kBLayout);
+                            mma_bf16(d, adesc, bdesc, idesc, (c > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        mma_commit(emptyA0 + 8 * ws);
+                        mma_commit(emptyA0 + 8 * as);
+                    }
+                    if (aborted) break;
+                    jb = jn;
+                    continue;
+                }
+                const int gw = (j - ncj) & (kGatherWarps - 1);
                 int bs = job_bslot(jb);
                 uint32_t bph = job_bphase(jb);
                 for (int c = 0; c < nchunks; ++c) {
@@ -430,22 +491,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         // up once and serve every channel chunk.  Each lane arrives on the slot's
         // barrier when its own copies land (cp.async.mbarrier.arrive.noinc), so no
         // producer ever waits for data.
-        const int gw = warp - kWarpGather0;
+        const int gw = warp == 0 ? 0 : warp - 1;
         const int q = lane % L::kThreadsPerRow;
         const int prow = lane / L::kThreadsPerRow;
         const int atom = q / L::kChunksPerAtom, qa = q % L::kChunksPerAtom;
         int s = 0;
         uint32_t ph = 0;
-        for (int j = gw; j < njobs && !aborted; j += kGatherWarps) {
+        for (int j = ncj + gw; j < njobs && !aborted; j += kGatherWarps) {
             const int4 jb = jobs[j];
-            const bool centre = job_centre(jb);
             const int n = jb.z, ncols = jb.w;
             int src[L::kPasses];
 #pragma unroll
             for (int ps = 0; ps < L::kPasses; ++ps) {
                 const int pr = prow + ps * L::kWarpRows;
-                src[ps] = -1;
-                if (pr < n) src[ps] = centre ? (int)row0 + jb.y + pr : pj_s[jb.y + pr];
+                src[ps] = pr < n ? pj_s[jb.y + pr] : -1;
             }
             for (int c = 0; c < nchunks; ++c) {
                 const int slot = gw * SB + s;
@@ -621,6 +680,21 @@ spconv_status_t launch(const MapData& m, const void* x, int cin, const void* w, 
         *ce = cudaErrorInvalidValue;
         return SPCONV_ERR_CUDA;
     }
+    // Features [n, cin] for the centre jobs: a box is one swizzle atom of channels
+    // by BM rows.
+    CUtensorMap xm;
+    const cuuint64_t xdims[2] = {(cuuint64_t)cin, (cuuint64_t)m.n};
+    const cuuint64_t xstrides[1] = {(cuuint64_t)cin * 2};
+    const cuuint32_t xbox[2] = {(cuuint32_t)L::kAtomElems, (cuuint32_t)BM};
+    const CUtensorMapSwizzle xswz = L::kAtomRowBytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                    : L::kAtomRowBytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                             : CU_TENSOR_MAP_SWIZZLE_32B;
+    r = enc(&xm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), xdims, xstrides, xbox, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, xswz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        *ce = cudaErrorInvalidValue;
+        return SPCONV_ERR_CUDA;
+    }
     const int smem = L::smem_bytes(cap, sa, sb);
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
@@ -648,7 +722,7 @@ spconv_status_t launch(const MapData& m, const void* x, int cin, const void* w, 
     p.sb = sb;
     p.cap = cap;
     dim3 grid((unsigned)((m.n + kTileRows - 1) / kTileRows), (unsigned)((cout + BM - 1) / BM));
-    k_subm_tc<BM, KC><<<grid, kThreads, smem, stream>>>(map, p);
+    k_subm_tc<BM, KC><<<grid, kThreads, smem, stream>>>(map, xm, p);
     *ce = cudaGetLastError();
     return *ce == cudaSuccess ? SPCONV_OK : SPCONV_ERR_CUDA;
 }

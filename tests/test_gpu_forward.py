@@ -69,7 +69,7 @@ def test_bf16_tcgen05_matches_oracle(sp, cin, cout, bias):
     assert_close(out, _ref(coords, ext, x, w, b), "bf16")
 
 
-@pytest.mark.parametrize("cin,cout", [(64, 64), (128, 128), (512, 512), (32, 64)])
+@pytest.mark.parametrize("cin,cout", [(64, 64), (128, 128), (512, 512), (32, 64), (16, 64), (48, 128)])
 def test_bf16_kernel_size_one(sp, cin, cout):
     coords, ext, x, w, b = _case(2, 30, 1500, cin, cout, kvol=1)
     out = _run(sp, coords, ext, x, w, b, "bf16", algo=sp.ALGO_TCGEN05)
