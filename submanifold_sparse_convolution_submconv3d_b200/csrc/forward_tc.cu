@@ -166,7 +166,7 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 1;; ++i) {
         if (kSpin ? mbar_test_wait(bar, parity) : mbar_try_wait_hint(bar, parity, kSuspendHintNs)) return true;
-        if (kSpin && (i & 255) != 0) continue;
+        if ((i & (kSpin ? 255u : 15u)) != 0) continue;  // the timer and the abort flag every few polls
         if (*abort_flag) return false;
         if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
             *abort_flag = 1;
