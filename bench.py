@@ -136,6 +136,24 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest of every rank's x (the slowest rank sets a multi-GPU time);
+    every rank must call it, in the same order."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_mvox(world: int, steps: int, layers: int, n: int, total_ms: float) -> float:
+    """Whole-job throughput in Mvox/s per layer: every rank processes its own copy
+    of the n-voxel workload (replicas), so the units add up over ranks."""
+    return world * steps * layers * n / (total_ms / 1e3) / 1e6
+
+
 def roofline_bytes_flops(n: int, pairs: int, cin: int, cout: int) -> tuple[float, float]:
     """Compulsory bytes and useful FLOPs of one k=3 layer: x read once, W once, bias,
     out written once, 4 bytes per non-centre neighbour pair; 2*Cin*Cout per pair."""
@@ -253,11 +271,8 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     clocks = sampler.stop()
     m.check()
     total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-    value = world * args.steps * LAYERS * n / (total_ms / 1e3) / 1e6
+    total_ms = max_over_ranks(total_ms, world, dev)
+    value = whole_job_mvox(world, args.steps, LAYERS, n, total_ms)
 
     # ---- map build, timed separately (pack + insert + probe, one host sync inside)
     build_ms = []
@@ -293,11 +308,8 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         if i >= args.warmup:
             e2e_ms.append(dt)
     e2e_total = sum(e2e_ms)
-    if world > 1:
-        t = torch.tensor([e2e_total], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_total = float(t.item())
-    e2e_value = world * args.steps * LAYERS * n / (e2e_total / 1e3) / 1e6
+    e2e_total = max_over_ranks(e2e_total, world, dev)
+    e2e_value = whole_job_mvox(world, args.steps, LAYERS, n, e2e_total)
 
     if rank != 0:
         return
