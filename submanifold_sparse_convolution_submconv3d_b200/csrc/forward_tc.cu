@@ -25,8 +25,9 @@
 // centre job).  At the end each output row is written exactly once, with bias,
 // rounded to bf16.
 //
-// Warp roles (576 threads):
-//   warp 1      TMEM allocator and tcgen05.mma issuer
+// Warp roles (608 threads):
+//   warps 1, 18 TMEM allocator (warp 1) and the two tcgen05.mma issuers, which
+//               take alternate jobs
 //   warp 5      TMA producer of weight tiles (A operand), a ring of 2-6 slots
 //   warps 0, 2-4  gather producers (B operand): gather warp g fills the jobs j
 //               with j % 4 == g into its own ring of slots, in order, so each
@@ -62,9 +63,9 @@ static_assert(kDummyCol0 + 16 <= kTmemCols, "accumulator, scratch buffers and du
 // sub-partition of its TMEM lane quarter.  The MMA issuer's sub-partition (1)
 // therefore hosts, besides three fold warps, only the light weight producer; the
 // four gather warps (0, 2, 3, 4) go to the others.
-constexpr int kWarpMma = 1, kWarpTma = 5, kWarpFold0 = 6;
+constexpr int kWarpMma = 1, kWarpTma = 5, kWarpFold0 = 6, kWarpMma2 = 18;
 constexpr int kGatherWarps = 4, kFoldWarps = 12;
-constexpr int kThreads = 32 * (kWarpFold0 + kFoldWarps);  // 576
+constexpr int kThreads = 32 * (kWarpFold0 + kFoldWarps + 1);  // 608
 constexpr int kFoldGroup = 16;
 constexpr int kMaxASlots = 6;                             // weight ring slots
 constexpr int kMaxBSlots = 8;                             // gather ring slots per gather warp
@@ -114,7 +115,7 @@ struct Layout {
     static constexpr int kFixedMeta = kMaxJobs * 16 + 2 * kTileCountStride * 4;
 
     __host__ __device__ static int ring_bytes(int sa, int sb) { return sa * kAPad + kGatherWarps * sb * kBPad; }
-    __host__ __device__ static int num_bars(int sa, int sb) { return 2 * sa + 2 * kGatherWarps * sb + 2 * kScratchBufs + 2; }
+    __host__ __device__ static int num_bars(int sa, int sb) { return 2 * sa + 2 * kGatherWarps * sb + 2 * kScratchBufs + 4; }
     __host__ __device__ static int smem_bytes(int cap, int sa, int sb) {
         return 1024 + ring_bytes(sa, sb) + kFixedMeta + cap * 4 + round_up(cap * 2, 16) + num_bars(sa, sb) * 8 + 16;
     }
@@ -211,7 +212,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t fullA0 = smem_addr(bars), emptyA0 = fullA0 + 8 * SA;
     const uint32_t fullB0 = emptyA0 + 8 * SA, emptyB0 = fullB0 + 8 * kGatherWarps * SB;
     const uint32_t sfull0 = emptyB0 + 8 * kGatherWarps * SB, sempty0 = sfull0 + 8 * kScratchBufs;
-    const uint32_t accfull = sempty0 + 8 * kScratchBufs, drain = accfull + 8;
+    const uint32_t accfull = sempty0 + 8 * kScratchBufs, drain0 = accfull + 8;  // drain0, drain1: one per issuer
+    const uint32_t centre_done = drain0 + 16;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t row0 = (int64_t)blockIdx.x * kTileRows;
@@ -223,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < SA; ++s) {
             mbar_init(fullA0 + 8 * s, 1);
-            mbar_init(emptyA0 + 8 * s, 1);
+            mbar_init(emptyA0 + 8 * s, 2);  // both issuers release every weight-ring use
         }
         for (int s = 0; s < kGatherWarps * SB; ++s) {
             mbar_init(fullB0 + 8 * s, 32);  // the 32 lanes of the filling gather warp
@@ -233,8 +235,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(sfull0 + 8 * b, 1);
             mbar_init(sempty0 + 8 * b, kFoldWarps);
         }
-        mbar_init(accfull, 1);
-        mbar_init(drain, 1);
+        mbar_init(accfull, 2);
+        mbar_init(drain0, 1);
+        mbar_init(drain0 + 8, 1);
+        mbar_init(centre_done, 2);
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tensormap(&wmap);
@@ -368,29 +372,38 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (aborted) __nanosleep(200000);  // let loads in flight land before the CTA exits
         }
-    } else if (warp == kWarpMma) {
-        // ------------------------------------------------ tcgen05.mma issuer
+    } else if (warp == kWarpMma || warp == kWarpMma2) {
+        // ------------------------------------------------ tcgen05.mma issuers
+        // Two issuer threads take alternate jobs (issuer me owns the jobs j with
+        // j % 2 == me), so one's bookkeeping and waits overlap the other's MMAs.
+        //  * Weight ring: both walk every ring use in order, wait for it to fill and
+        //    commit its release once (the slot's empty barrier counts two), so no
+        //    issuer can run a ring length ahead of the other.
+        //  * Gather rings: offset job ncj + q comes from gather warp q % 4, and
+        //    (ncj + q) % 2 = me keeps each gather warp's jobs with one issuer.
+        //  * Scratch buffers: offset job ncj + q uses buffer q % 2, so each issuer
+        //    owns one buffer and uses it in order.
+        //  * The fold starts after both issuers' centre MMAs (centre_done).
         if (lane == 0) {
-            int as = SA - 1, prev_k = -1;  // weight slot in use and its phase
+            const int me = warp == kWarpMma ? 0 : 1;
+            const int own_b = (me + ncj) & 1;  // this issuer's scratch buffer
+            uint32_t own_ph = 1u;              // parity of its previous use
+            int as = SA - 1, prev_k = -1;      // weight slot in use and its phase
             uint32_t aph = 1u;
-            int sb_ = kScratchBufs - 1;  // scratch buffer of the last offset job and its phase
-            uint32_t sph = 1u;
             int4 jb = njobs > 0 ? jobs[0] : make_int4(0, 0, 0, 0);
             for (int j = 0; j < njobs && !aborted; ++j) {
                 const int4 jn = j + 1 < njobs ? jobs[j + 1] : make_int4(-1, 0, 0, 0);  // prefetch
                 const int k = job_k(jb);
                 const bool centre = job_centre(jb);
+                const bool mine = (j & 1) == me;
                 const bool new_k = k != prev_k;
                 prev_k = k;
                 const bool last_of_k = j + 1 == njobs || job_k(jn) != k;
                 uint32_t d = tmem + (uint32_t)jb.y;
-                if (!centre) {
-                    if (++sb_ == kScratchBufs) {
-                        sb_ = 0;
-                        sph ^= 1u;
-                    }
-                    d = tmem + kScratchCol0 + (uint32_t)sb_ * kJobRows;
-                    if (!wait_bar(sempty0 + 8 * sb_, sph ^ 1u, abort_flag, p.err)) {
+                if (mine && !centre) {
+                    own_ph ^= 1u;
+                    d = tmem + kScratchCol0 + (uint32_t)own_b * kJobRows;
+                    if (!wait_bar(sempty0 + 8 * own_b, own_ph ^ 1u, abort_flag, p.err)) {
                         aborted = true;
                         break;
                     }
@@ -413,21 +426,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                         }
                         if (aborted) break;
-                        const uint32_t a_base = smem_addr(a_ring + ws * L::kAPad);
-                        const uint32_t x_base = smem_addr(a_ring + as * L::kAPad);
+                        if (mine) {
+                            const uint32_t a_base = smem_addr(a_ring + ws * L::kAPad);
+                            const uint32_t x_base = smem_addr(a_ring + as * L::kAPad);
 #pragma unroll
-                        for (int kk = 0; kk < KC / 16; ++kk) {
-                            const uint64_t adesc = smem_desc(a_base + kk * 2048, KC * 128, 1024, 2);
-                            constexpr int kStepsPerAtom = L::kAtomElems / 16;
-                            const uint64_t bdesc = smem_desc(
-                                x_base + (kk / kStepsPerAtom) * (BM * L::kAtomRowBytes) + (kk % kStepsPerAtom) * 32, 16,
-                                L::kBSbo, L::kBLayout);
-                            mma_bf16(d, adesc, bdesc, idesc, (c > 0 || kk > 0) ? 1u : 0u);
+                            for (int kk = 0; kk < KC / 16; ++kk) {
+                                const uint64_t adesc = smem_desc(a_base + kk * 2048, KC * 128, 1024, 2);
+                                constexpr int kStepsPerAtom = L::kAtomElems / 16;
+                                const uint64_t bdesc = smem_desc(
+                                    x_base + (kk / kStepsPerAtom) * (BM * L::kAtomRowBytes) + (kk % kStepsPerAtom) * 32,
+                                    16, L::kBSbo, L::kBLayout);
+                                mma_bf16(d, adesc, bdesc, idesc, (c > 0 || kk > 0) ? 1u : 0u);
+                            }
                         }
                         mma_commit(emptyA0 + 8 * ws);
                         mma_commit(emptyA0 + 8 * as);
                     }
                     if (aborted) break;
+                    if (j == ncj - 1) mma_commit(centre_done);
                     jb = jn;
                     continue;
                 }
@@ -445,40 +461,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                             break;
                         }
                     }
-                    const int bslot = gw * SB + bs;
-                    if (!wait_bar(fullB0 + 8 * bslot, bph, abort_flag, p.err)) {
-                        aborted = true;
-                        break;
-                    }
-                    // the B tile was written by cp.async (generic proxy); the MMA reads it
-                    // through the async proxy
-                    fence_proxy_async_smem();
-                    const uint32_t a_base = smem_addr(a_ring + as * L::kAPad);
-                    const uint32_t b_base = smem_addr(b_ring + bslot * L::kBPad);
+                    if (mine) {
+                        const int bslot = gw * SB + bs;
+                        if (!wait_bar(fullB0 + 8 * bslot, bph, abort_flag, p.err)) {
+                            aborted = true;
+                            break;
+                        }
+                        // the B tile was written by cp.async (generic proxy); the MMA reads it
+                        // through the async proxy
+                        fence_proxy_async_smem();
+                        const uint32_t a_base = smem_addr(a_ring + as * L::kAPad);
+                        const uint32_t b_base = smem_addr(b_ring + bslot * L::kBPad);
 #pragma unroll
-                    for (int kk = 0; kk < KC / 16; ++kk) {
-                        const uint64_t adesc = smem_desc(a_base + kk * 2048, KC * 128, 1024, 2);
-                        constexpr int kStepsPerAtom = L::kAtomElems / 16;
-                        const uint64_t bdesc =
-                            smem_desc(b_base + (kk / kStepsPerAtom) * L::kBAtomBytes + (kk % kStepsPerAtom) * 32, 16,
-                                      L::kBSbo, L::kBLayout);
-                        mma_bf16(d, adesc, bdesc, idesc, (c > 0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < KC / 16; ++kk) {
+                            const uint64_t adesc = smem_desc(a_base + kk * 2048, KC * 128, 1024, 2);
+                            constexpr int kStepsPerAtom = L::kAtomElems / 16;
+                            const uint64_t bdesc =
+                                smem_desc(b_base + (kk / kStepsPerAtom) * L::kBAtomBytes + (kk % kStepsPerAtom) * 32,
+                                          16, L::kBSbo, L::kBLayout);
+                            mma_bf16(d, adesc, bdesc, idesc, (c > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        mma_commit(emptyB0 + 8 * bslot);
+                        if (++bs == SB) {
+                            bs = 0;
+                            bph ^= 1u;
+                        }
                     }
-                    mma_commit(emptyB0 + 8 * bslot);
                     if (nchunks > 1 || last_of_k) mma_commit(emptyA0 + 8 * as);
-                    if (++bs == SB) {
-                        bs = 0;
-                        bph ^= 1u;
-                    }
                 }
                 if (aborted) break;
-                if (!centre) mma_commit(sfull0 + 8 * sb_);
+                if (mine) mma_commit(sfull0 + 8 * own_b);
                 jb = jn;
             }
             if (!aborted) {
                 mma_commit(accfull);
             } else {
-                mma_commit(drain);  // wait for MMAs in flight before TMEM is freed
+                const uint32_t drain = drain0 + 8 * me;
+                mma_commit(drain);  // wait for this issuer's MMAs in flight before TMEM is freed
                 const uint64_t t0 = globaltimer_ns();
                 while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
                 }
@@ -532,7 +551,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         cp_async_wait_all();
-    } else {
+    } else if (warp < kWarpFold0 + kFoldWarps) {
         // ------------------------------------------------ fold scratch -> accumulator, then epilogue
         // Warp (quarter, sub) owns TMEM lanes [32*quarter, +32) and the tile rows
         // r with r % 3 == sub, so every accumulator column is only ever touched by
@@ -542,7 +561,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
         int b = kScratchBufs - 1;  // scratch buffer of the current offset job and its phase
         uint32_t sph = 1u;
-        for (int j = 0; j < njobs; ++j) {
+        // both issuers' centre MMAs write accumulator columns: they complete first
+        if (warp_wait_bar(centre_done, 0, abort_flag, p.err))
+            tc_fence_after();
+        else
+            aborted = true;
+        for (int j = 0; j < njobs && !aborted; ++j) {
             const int4 jb = jobs[j];
             if (job_centre(jb)) continue;
             if (++b == kScratchBufs) {
