@@ -156,6 +156,15 @@ SPCONV_API spconv_status_t spconv_subm_forward_algo(spconv_map_t map, spconv_dty
 SPCONV_API spconv_status_t spconv_debug_set_table_slots(int64_t slots);
 
 /*
+ * Test hook: force the tile height (rows per forward CTA, 1..384) of later builds
+ * in this process; 0 restores the automatic choice, the smallest height that
+ * fills the same number of waves of SMs as 384-row tiles.  Lets tests run small
+ * inputs through full-height tiles (several jobs per offset).  Other values:
+ * SPCONV_ERR_INVALID_ARG.
+ */
+SPCONV_API spconv_status_t spconv_debug_set_tile_rows(int32_t rows);
+
+/*
  * Neighbour-map build that allocates no device memory.  The pages have no
  * counterpart: this is an interface for callers that cannot call cudaMalloc or
  * cudaFree -- code running while another component owns the device memory (a

@@ -27,7 +27,7 @@ _DTYPES = {torch.float32: 0, torch.bfloat16: 1}
 
 EXPORTED = ("spconv_build_map", "spconv_subm_forward", "spconv_free", "spconv_map_info", "spconv_map_check",
             "spconv_last_error", "spconv_subm_forward_algo", "spconv_debug_set_table_slots",
-            "spconv_build_neighbor_map_noalloc")
+            "spconv_debug_set_tile_rows", "spconv_build_neighbor_map_noalloc")
 
 
 class SpconvError(RuntimeError):
@@ -50,11 +50,12 @@ def _load() -> ctypes.CDLL:
                                     ctypes.POINTER(vp)]
     lib.spconv_map_check.argtypes = [vp, vp]
     lib.spconv_debug_set_table_slots.argtypes = [i64]
+    lib.spconv_debug_set_tile_rows.argtypes = [i32]
     lib.spconv_build_neighbor_map_noalloc.argtypes = [vp, i64, vp, vp, ctypes.POINTER(i64), vp]
     lib.spconv_last_error.restype = ctypes.c_char_p
     for name in ("spconv_build_map", "spconv_subm_forward", "spconv_subm_forward_algo", "spconv_free",
                  "spconv_map_info", "spconv_map_check", "spconv_debug_set_table_slots",
-                 "spconv_build_neighbor_map_noalloc"):
+                 "spconv_debug_set_tile_rows", "spconv_build_neighbor_map_noalloc"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -199,7 +200,13 @@ def spconv_debug_set_table_slots(slots: int) -> None:
     _check(lib.spconv_debug_set_table_slots(int(slots)))
 
 
+def spconv_debug_set_tile_rows(rows: int) -> None:
+    _require()
+    _check(lib.spconv_debug_set_tile_rows(int(rows)))
+
+
 __all__ = ["OK", "INVALID_ARG", "UNSUPPORTED", "COORD_RANGE", "DUPLICATE", "TABLE_FULL", "OOM", "CUDA_ERROR",
            "TIMEOUT", "SubmMap", "SpconvError", "spconv_build_map", "spconv_subm_forward", "spconv_free",
-           "spconv_debug_set_table_slots", "spconv_build_neighbor_map_noalloc", "lib", "LIB_PATH", "EXPORTED",
+           "spconv_debug_set_table_slots", "spconv_debug_set_tile_rows", "spconv_build_neighbor_map_noalloc", "lib",
+           "LIB_PATH", "EXPORTED",
            "ALGO_AUTO", "ALGO_SIMT", "ALGO_TCGEN05"]

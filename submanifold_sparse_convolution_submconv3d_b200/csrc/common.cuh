@@ -34,7 +34,8 @@ constexpr int kVol3 = 27;
 constexpr int kCentre = 13;
 
 // Tile metadata (built with the map, kernel size 3): the rows are cut into tiles
-// of kTileRows consecutive rows; for every tile and every non-centre offset the
+// of `tile_rows` consecutive rows (at most kTileRows, chosen per map by
+// choose_tile_rows); for every tile and every non-centre offset the
 // tile rows with an active neighbour there are listed, split into three classes
 // by row % 3 and sorted by row within a class.  "Units" are (offset, class)
 // pairs in offset-major order, offsets 0..26 without the centre: unit
@@ -45,7 +46,18 @@ constexpr int kTileUnits = (kVol3 - 1) * kTileClasses;  // 78
 constexpr int kTileCountStride = 80;                    // int32 counts per tile (78 used), 320 bytes
 constexpr int kTileEntryAlign = 8;                      // each tile's entries start on a multiple of 8
 
-__host__ __device__ inline int64_t num_tiles(int64_t n) { return (n + kTileRows - 1) / kTileRows; }
+__host__ __device__ inline int64_t num_tiles(int64_t n, int tile_rows) { return (n + tile_rows - 1) / tile_rows; }
+
+// Rows per tile for n voxels on num_sms SMs (one tile per SM at a time): the
+// number of waves that kTileRows-row tiles need, then the smallest tile that
+// still fits n into that many waves, so the last wave is not left mostly empty.
+inline int choose_tile_rows(int64_t n, int num_sms) {
+    if (n <= 0 || num_sms <= 0) return kTileRows;
+    const int64_t per_wave = (int64_t)kTileRows * num_sms;
+    const int64_t waves = (n + per_wave - 1) / per_wave;
+    const int64_t rows = (n + waves * num_sms - 1) / (waves * num_sms);
+    return (int)(rows < 32 ? (n < 32 ? n : 32) : rows);
+}
 
 // The map handle (defined here so the launchers can read it).
 struct MapData {
@@ -63,6 +75,7 @@ struct MapData {
     int32_t* pair_j = nullptr;
     int64_t tile_entries = 0;
     int64_t tile_max_entries = 0;  // entries of the fullest tile (a multiple of kTileEntryAlign)
+    int32_t tile_rows = kTileRows;  // rows per tile (<= kTileRows), for the forward kernels too
     unsigned int* fwd_err = nullptr;  // device word: forward-kernel error bits
     int device = 0;
     int num_sms = 0;
@@ -78,10 +91,10 @@ cudaError_t launch_build_map(const int32_t* coords, int64_t n, const int32_t ext
 
 // Tile metadata in two passes: counts + offsets (then the caller reads the total
 // and allocates the entry arrays), then the entries.
-cudaError_t launch_tile_count(const int32_t* nbr, int64_t n, int32_t* tile_counts, int64_t* tile_off,
+cudaError_t launch_tile_count(const int32_t* nbr, int64_t n, int tile_rows, int32_t* tile_counts, int64_t* tile_off,
                               cudaStream_t stream);
-cudaError_t launch_tile_fill(const int32_t* nbr, int64_t n, const int32_t* tile_counts, const int64_t* tile_off,
-                             uint16_t* pair_r, int32_t* pair_j, cudaStream_t stream);
+cudaError_t launch_tile_fill(const int32_t* nbr, int64_t n, int tile_rows, const int32_t* tile_counts,
+                             const int64_t* tile_off, uint16_t* pair_r, int32_t* pair_j, cudaStream_t stream);
 
 cudaError_t launch_forward_simt(const MapData& m, spconv_dtype_t dtype, const void* x, int cin, const void* w,
                                 const void* bias, void* out, int cout, cudaStream_t stream);

@@ -7,7 +7,8 @@
 //
 //   D^T[Cout_blk, rows] = sum_k W_k^T[Cout_blk, Cin] . X_k^T[Cin, rows]
 //
-// One CTA owns kTileRows consecutive output rows and one block of 64 or 128
+// One CTA owns a tile of consecutive output rows (at most kTileRows, chosen per
+// map so that the tiles fill whole waves of SMs) and one block of 64 or 128
 // output channels.  Tensor memory (TMEM, 128 lanes x 512 fp32 columns) holds
 //   * the accumulator: lane = output channel, column = output row of the tile;
 //   * two scratch buffers of kJobRows columns and 16 dummy columns.
@@ -152,6 +153,7 @@ struct Params {
     __nv_bfloat16* out;
     int cout;
     unsigned int* err;
+    int tile_rows;  // rows per tile (<= kTileRows)
     int sa;   // weight ring slots
     int sb;   // gather slots per gather warp
     int cap;  // entry capacity of the shared-memory lists (largest tile's entries)
@@ -216,8 +218,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t centre_done = drain0 + 16;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t row0 = (int64_t)blockIdx.x * kTileRows;
-    const int t_eff = (int)min((int64_t)kTileRows, p.n - row0);
+    const int64_t row0 = (int64_t)blockIdx.x * p.tile_rows;
+    const int t_eff = (int)min((int64_t)p.tile_rows, p.n - row0);
     const int cblk = blockIdx.y;
     const int nchunks = p.cin / KC;
 
@@ -742,10 +744,11 @@ spconv_status_t launch(const MapData& m, const void* x, int cin, const void* w, 
     p.out = static_cast<__nv_bfloat16*>(out);
     p.cout = cout;
     p.err = m.fwd_err;
+    p.tile_rows = m.tile_rows;
     p.sa = sa;
     p.sb = sb;
     p.cap = cap;
-    dim3 grid((unsigned)((m.n + kTileRows - 1) / kTileRows), (unsigned)((cout + BM - 1) / BM));
+    dim3 grid((unsigned)num_tiles(m.n, m.tile_rows), (unsigned)((cout + BM - 1) / BM));
     k_subm_tc<BM, KC><<<grid, kThreads, smem, stream>>>(map, xm, p);
     *ce = cudaGetLastError();
     return *ce == cudaSuccess ? SPCONV_OK : SPCONV_ERR_CUDA;

@@ -143,13 +143,13 @@ __device__ __forceinline__ int unit_offset(int u) {
     return ks < kCentre ? ks : ks + 1;
 }
 
-__global__ void k_tile_count(const int32_t* __restrict__ nbr, int64_t n, int32_t* __restrict__ tile_counts,
-                             int64_t* __restrict__ tile_total) {
+__global__ void k_tile_count(const int32_t* __restrict__ nbr, int64_t n, int tile_rows,
+                             int32_t* __restrict__ tile_counts, int64_t* __restrict__ tile_total) {
     __shared__ int32_t tile_s[kTileRows * kVol3];
     __shared__ int32_t cnt_s[kTileUnits];
     const int64_t t = blockIdx.x;
-    const int64_t row0 = t * kTileRows;
-    const int t_eff = (int)min((int64_t)kTileRows, n - row0);
+    const int64_t row0 = t * tile_rows;
+    const int t_eff = (int)min((int64_t)tile_rows, n - row0);
     stage_tile_rows(nbr, row0, t_eff, tile_s);
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -209,14 +209,15 @@ __global__ void k_tile_scan(int64_t* __restrict__ off, int64_t ntiles) {
     }
 }
 
-__global__ void k_tile_fill(const int32_t* __restrict__ nbr, int64_t n, const int32_t* __restrict__ tile_counts,
+__global__ void k_tile_fill(const int32_t* __restrict__ nbr, int64_t n, int tile_rows,
+                            const int32_t* __restrict__ tile_counts,
                             const int64_t* __restrict__ tile_off, uint16_t* __restrict__ pair_r,
                             int32_t* __restrict__ pair_j) {
     __shared__ int32_t tile_s[kTileRows * kVol3];
     __shared__ int32_t start_s[kTileUnits];
     const int64_t t = blockIdx.x;
-    const int64_t row0 = t * kTileRows;
-    const int t_eff = (int)min((int64_t)kTileRows, n - row0);
+    const int64_t row0 = t * tile_rows;
+    const int t_eff = (int)min((int64_t)tile_rows, n - row0);
     stage_tile_rows(nbr, row0, t_eff, tile_s);
     if (threadIdx.x == 0) {
         int run = 0;
@@ -253,22 +254,24 @@ __global__ void k_tile_fill(const int32_t* __restrict__ nbr, int64_t n, const in
 
 }  // namespace
 
-cudaError_t launch_tile_count(const int32_t* nbr, int64_t n, int32_t* tile_counts, int64_t* tile_off,
+cudaError_t launch_tile_count(const int32_t* nbr, int64_t n, int tile_rows, int32_t* tile_counts, int64_t* tile_off,
                               cudaStream_t stream) {
-    const int64_t nt = num_tiles(n);
+    if (tile_rows < 1 || tile_rows > kTileRows) return cudaErrorInvalidValue;
+    const int64_t nt = num_tiles(n, tile_rows);
     if (nt == 0) return cudaMemsetAsync(tile_off, 0, 2 * sizeof(int64_t), stream);
-    k_tile_count<<<(unsigned)nt, kMetaThreads, 0, stream>>>(nbr, n, tile_counts, tile_off);
+    k_tile_count<<<(unsigned)nt, kMetaThreads, 0, stream>>>(nbr, n, tile_rows, tile_counts, tile_off);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     k_tile_scan<<<1, 1024, 0, stream>>>(tile_off, nt);
     return cudaGetLastError();
 }
 
-cudaError_t launch_tile_fill(const int32_t* nbr, int64_t n, const int32_t* tile_counts, const int64_t* tile_off,
-                             uint16_t* pair_r, int32_t* pair_j, cudaStream_t stream) {
-    const int64_t nt = num_tiles(n);
+cudaError_t launch_tile_fill(const int32_t* nbr, int64_t n, int tile_rows, const int32_t* tile_counts,
+                             const int64_t* tile_off, uint16_t* pair_r, int32_t* pair_j, cudaStream_t stream) {
+    if (tile_rows < 1 || tile_rows > kTileRows) return cudaErrorInvalidValue;
+    const int64_t nt = num_tiles(n, tile_rows);
     if (nt == 0) return cudaSuccess;
-    k_tile_fill<<<(unsigned)nt, kMetaThreads, 0, stream>>>(nbr, n, tile_counts, tile_off, pair_r, pair_j);
+    k_tile_fill<<<(unsigned)nt, kMetaThreads, 0, stream>>>(nbr, n, tile_rows, tile_counts, tile_off, pair_r, pair_j);
     return cudaGetLastError();
 }
 

@@ -12,6 +12,7 @@ namespace {
 
 thread_local std::string g_last_error;
 int64_t g_table_slots_override = 0;
+int32_t g_tile_rows_override = 0;
 
 spconv_status_t fail(spconv_status_t s, const std::string& msg) {
     g_last_error = msg;
@@ -44,6 +45,12 @@ const char* spconv_last_error(void) { return g_last_error.c_str(); }
 spconv_status_t spconv_debug_set_table_slots(int64_t slots) {
     if (slots < 0 || (slots & (slots - 1)) != 0) return fail(SPCONV_ERR_INVALID_ARG, "slots must be 0 or a power of two");
     g_table_slots_override = slots;
+    return SPCONV_OK;
+}
+
+spconv_status_t spconv_debug_set_tile_rows(int32_t rows) {
+    if (rows < 0 || rows > spconv::kTileRows) return fail(SPCONV_ERR_INVALID_ARG, "rows must be in [0, 384]");
+    g_tile_rows_override = rows;
     return SPCONV_OK;
 }
 
@@ -82,13 +89,15 @@ spconv_status_t spconv_build_map(const int32_t* coords, int64_t n, const int32_t
     e = cudaMalloc(&table, slots * 16);
     if (e == cudaSuccess) e = cudaMalloc(&flags, sizeof(spconv::BuildFlags));
     if (e == cudaSuccess && kernel_size == 3 && n > 0) e = cudaMalloc(&m->d.nbr, (size_t)n * spconv::kVol3 * sizeof(int32_t));
-    const int64_t ntiles = spconv::num_tiles(n);
+    m->d.tile_rows = g_tile_rows_override > 0 ? g_tile_rows_override : spconv::choose_tile_rows(n, m->d.num_sms);
+    const int64_t ntiles = spconv::num_tiles(n, m->d.tile_rows);
     const bool tiles = kernel_size == 3 && n > 0;
     if (e == cudaSuccess && tiles) e = cudaMalloc(&m->d.tile_counts, (size_t)ntiles * spconv::kTileCountStride * 4);
     if (e == cudaSuccess && tiles) e = cudaMalloc(&m->d.tile_off, (size_t)(ntiles + 2) * sizeof(int64_t));
     if (e == cudaSuccess)
         e = spconv::launch_build_map(coords, n, extent, kernel_size, table, slots, m->d.nbr, flags, stream);
-    if (e == cudaSuccess && tiles) e = spconv::launch_tile_count(m->d.nbr, n, m->d.tile_counts, m->d.tile_off, stream);
+    if (e == cudaSuccess && tiles)
+        e = spconv::launch_tile_count(m->d.nbr, n, m->d.tile_rows, m->d.tile_counts, m->d.tile_off, stream);
     int64_t entry_stats[2] = {0, 0};  // grand total, largest tile
     if (e == cudaSuccess && tiles)
         e = cudaMemcpyAsync(entry_stats, m->d.tile_off + ntiles, sizeof(entry_stats), cudaMemcpyDeviceToHost, stream);
@@ -103,8 +112,8 @@ spconv_status_t spconv_build_map(const int32_t* coords, int64_t n, const int32_t
         e = cudaMalloc(&m->d.pair_r, ne * sizeof(uint16_t));
         if (e == cudaSuccess) e = cudaMalloc(&m->d.pair_j, ne * sizeof(int32_t));
         if (e == cudaSuccess)
-            e = spconv::launch_tile_fill(m->d.nbr, n, m->d.tile_counts, m->d.tile_off, m->d.pair_r, m->d.pair_j,
-                                         stream);
+            e = spconv::launch_tile_fill(m->d.nbr, n, m->d.tile_rows, m->d.tile_counts, m->d.tile_off, m->d.pair_r,
+                                         m->d.pair_j, stream);
         if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
     }
     if (e != cudaSuccess) {

@@ -57,7 +57,7 @@ def _case(seed, grid, n, cin, cout, kvol=27, bias=True):
     return coords, (grid,) * 3, x, w, b
 
 
-# Several 384-row tiles with a ragged tail; every kernel variant (Cout block 64 or
+# Several tiles with a ragged tail; every kernel variant (Cout block 64 or
 # 128; input chunk 16, 32 or 64 channels); with and without bias.
 @pytest.mark.parametrize("cin,cout,bias", [
     (64, 64, True), (128, 128, True), (128, 128, False), (32, 64, True), (16, 64, True),
@@ -110,6 +110,40 @@ def test_dense_block_and_isolated_voxels(sp):
     xi = workloads.round_to_bf16(rng.standard_normal((1000, 64), dtype=np.float32))
     out = _run(sp, iso, (64, 64, 64), xi, w[:, :, :64].copy(), b[:64].copy(), "bf16", algo=sp.ALGO_TCGEN05)
     assert_close(out, xi.astype(np.float64) @ w[13, :, :64] + b[:64], "bf16")
+
+
+@pytest.fixture
+def tile_rows(sp):
+    """Force the tile height of the maps a test builds; restores the automatic choice."""
+    def force(rows):
+        sp.spconv_debug_set_tile_rows(rows)
+    yield force
+    sp.spconv_debug_set_tile_rows(0)
+
+
+# Small inputs get short automatic tiles; the same cases through full-height
+# (384-row) tiles and an odd height exercise several jobs per offset, every
+# centre job of a tile and ragged tails inside a tile.
+@pytest.mark.parametrize("rows", [384, 100])
+@pytest.mark.parametrize("cin,cout,kvol", [(128, 128, 27), (64, 128, 27), (16, 64, 27), (512, 512, 27),
+                                           (128, 128, 1), (48, 128, 1)])
+def test_bf16_tcgen05_forced_tile_heights(sp, tile_rows, rows, cin, cout, kvol):
+    tile_rows(rows)
+    coords, ext, x, w, b = _case(9, 24, 2000, cin, cout, kvol=kvol)
+    out = _run(sp, coords, ext, x, w, b, "bf16", algo=sp.ALGO_TCGEN05)
+    assert_close(out, _ref(coords, ext, x, w, b), "bf16")
+
+
+def test_dense_block_full_height_tiles(sp, tile_rows):
+    rng = np.random.default_rng(11)
+    tile_rows(384)
+    blk = np.array([[0, a, b, c] for a in range(12) for b in range(12) for c in range(12)], np.int32)
+    blk = blk[rng.permutation(blk.shape[0])]
+    x = workloads.round_to_bf16(rng.standard_normal((blk.shape[0], 128), dtype=np.float32))
+    w = workloads.round_to_bf16(rng.standard_normal((27, 128, 128), dtype=np.float32) * 0.02)
+    b = workloads.round_to_bf16(rng.standard_normal(128, dtype=np.float32) * 0.1)
+    out = _run(sp, blk, (12, 12, 12), x, w, b, "bf16", algo=sp.ALGO_TCGEN05)
+    assert_close(out, _ref(blk, (12, 12, 12), x, w, b), "bf16")
 
 
 def test_single_voxel_and_single_tile_edge(sp):

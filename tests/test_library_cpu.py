@@ -61,6 +61,10 @@ def test_host_validation_without_device_work(pkg):
     assert lib.spconv_subm_forward(None, 1, None, 16, None, None, None, 16, None) == pkg.INVALID_ARG
     assert lib.spconv_debug_set_table_slots(3) == pkg.INVALID_ARG
     assert lib.spconv_debug_set_table_slots(0) == pkg.OK
+    assert lib.spconv_debug_set_tile_rows(-1) == pkg.INVALID_ARG
+    assert lib.spconv_debug_set_tile_rows(385) == pkg.INVALID_ARG
+    assert lib.spconv_debug_set_tile_rows(384) == pkg.OK
+    assert lib.spconv_debug_set_tile_rows(0) == pkg.OK
 
 
 def test_python_binding_rejects_bad_tensors(pkg):
