@@ -67,7 +67,8 @@ static_assert(kDummyCol0 + 16 <= kTmemCols, "accumulator, scratch buffers and du
 constexpr int kWarpMma = 1, kWarpTma = 5, kWarpFold0 = 6, kWarpMma2 = 18;
 constexpr int kGatherWarps = 4, kFoldWarps = 12;
 constexpr int kThreads = 32 * (kWarpFold0 + kFoldWarps + 1);  // 608
-constexpr int kFoldGroup = 16;
+constexpr int kFoldGroup = 16;    // scratch columns per wide TMEM load
+constexpr int kNarrowGroup = 16;  // accumulator columns per batch of narrow loads, then stores
 constexpr int kMaxASlots = 6;                             // weight ring slots
 constexpr int kMaxBSlots = 8;                             // gather ring slots per gather warp
 constexpr uint64_t kWaitTimeoutNs = 4000000000ull;
@@ -120,23 +121,26 @@ struct Layout {
     __host__ __device__ static int smem_bytes(int cap, int sa, int sb) {
         return 1024 + ring_bytes(sa, sb) + kFixedMeta + cap * 4 + round_up(cap * 2, 16) + num_bars(sa, sb) * 8 + 16;
     }
-    static bool fits(int cap, int sa, int sb) {
-        return smem_bytes(cap, sa, sb) <= kMaxSmem && ring_bytes(sa, sb) >= kOutStageBytes;
-    }
-    // Ring depths for a tile entry capacity `cap`: the deepest weight ring that
-    // fits beside one gather slot per warp (one job per offset is the common case,
-    // so most jobs wait on a fresh weight tile), then the room left to gather
-    // slots; {0, 0} if nothing fits.
+    static bool fits(int cap, int sa, int sb) { return smem_bytes(cap, sa, sb) <= kMaxSmem; }
+    // Ring depths for a tile entry capacity `cap`.  Gather depth matters more than
+    // weight depth (measured): keep three weight slots (two if nothing else fits;
+    // a centre job holds two at once), give the room to gather slots, then any
+    // room left back to weight slots.  The rings must also hold the epilogue's
+    // staging buffer.  {0, 0} if nothing fits.
     static void depths(int cap, int* sa, int* sb) {
         *sa = 0;
         *sb = 0;
-        int a = kMaxASlots;
-        while (a >= 2 && !fits(cap, a, 1)) --a;
-        if (a < 2) return;
-        int b = 1;
-        while (b < kMaxBSlots && fits(cap, a, b + 1)) ++b;
-        *sa = a;
-        *sb = b;
+        for (int a_min = 3; a_min >= 2; --a_min) {
+            if (!fits(cap, a_min, 1)) continue;
+            int b = 1;
+            while (b < kMaxBSlots && fits(cap, a_min, b + 1)) ++b;
+            int a = a_min;
+            while (a < kMaxASlots && fits(cap, a + 1, b)) ++a;
+            if (ring_bytes(a, b) < kOutStageBytes) continue;
+            *sa = a;
+            *sb = b;
+            return;
+        }
     }
 };
 
@@ -597,15 +601,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(sempty0 + 8 * b);
             // 2) then add them into the accumulator columns of their rows.
-            if (ng > 0) tmem_wait_st();  // this warp's stores of the previous job have landed
+            const int ngn = hi > lo ? (hi - lo + kNarrowGroup - 1) / kNarrowGroup : 0;
+            if (ngn > 0) tmem_wait_st();  // this warp's stores of the previous job have landed
 #pragma unroll
-            for (int gi = 0; gi < kJobRows / kFoldGroup; ++gi) {
-                if (gi < ng) {
-                    const int g0 = lo + gi * kFoldGroup;
-                    float a[kFoldGroup];
-                    uint32_t col[kFoldGroup];
+            for (int gi = 0; gi < kJobRows / kNarrowGroup; ++gi) {
+                if (gi < ngn) {
+                    const int g0 = lo + gi * kNarrowGroup;
+                    float a[kNarrowGroup];
+                    uint32_t col[kNarrowGroup];
 #pragma unroll
-                    for (int i = 0; i < kFoldGroup; ++i) {
+                    for (int i = 0; i < kNarrowGroup; ++i) {
                         const int e = g0 + i;
                         const uint32_t r = pr_s[min(e, hi - 1)];
                         col[i] = tmem + lane_base + (e < hi ? r : kDummyCol0 + (uint32_t)i);
@@ -613,7 +618,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < kFoldGroup; ++i) tmem_st_x1(col[i], a[i] + v[gi * kFoldGroup + i]);
+                    for (int i = 0; i < kNarrowGroup; ++i) tmem_st_x1(col[i], a[i] + v[gi * kNarrowGroup + i]);
                 }
             }
         }

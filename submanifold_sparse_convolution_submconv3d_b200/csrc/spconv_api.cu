@@ -202,7 +202,9 @@ spconv_status_t spconv_subm_forward_algo(spconv_map_t map, spconv_dtype_t dtype,
         if (s == SPCONV_OK) return SPCONV_OK;
         // The tensor-core kernel takes cout % 64 == 0; AUTO runs other bf16 shapes
         // on the CUDA-core kernel.
-        if (algo == SPCONV_ALGO_TCGEN05) return fail(s, "tcgen05 forward needs cout % 64 == 0");
+        if (algo == SPCONV_ALGO_TCGEN05)
+            return fail(s, "tcgen05 forward does not take this shape (cout % 64 != 0, cin % 16 != 0, or the tile lists "
+                           "do not fit shared memory)");
     }
     cudaError_t e = spconv::launch_forward_simt(map->d, dtype, x, cin, w, bias, out, cout, stream);
     if (e != cudaSuccess) return fail_cuda(e, "simt forward");
