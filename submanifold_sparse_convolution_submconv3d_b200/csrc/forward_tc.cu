@@ -68,7 +68,7 @@ constexpr int kWarpMma = 1, kWarpTma = 5, kWarpFold0 = 6, kWarpMma2 = 18;
 constexpr int kGatherWarps = 4, kFoldWarps = 12;
 constexpr int kThreads = 32 * (kWarpFold0 + kFoldWarps + 1);  // 608
 constexpr int kFoldGroup = 16;    // scratch columns per wide TMEM load
-constexpr int kNarrowGroup = 16;  // accumulator columns per batch of narrow loads, then stores
+constexpr int kNarrowGroup = 8;   // accumulator columns per batch of narrow loads, then stores
 constexpr int kMaxASlots = 6;                             // weight ring slots
 constexpr int kMaxBSlots = 8;                             // gather ring slots per gather warp
 constexpr uint64_t kWaitTimeoutNs = 4000000000ull;
