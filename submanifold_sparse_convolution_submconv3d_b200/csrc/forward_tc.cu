@@ -227,8 +227,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int cblk = blockIdx.y;
     const int nchunks = p.cin / KC;
 
-    // ---- set-up: barriers, TMEM, the tile's lists (cp.async, 16 B)
-    if (threadIdx.x == 0) {
+    // ---- set-up: barriers, TMEM, the tile's lists (cp.async, 16 B).  The weight
+    // producer initialises the barriers and at once issues the first two ring uses,
+    // which every tile has (centre weights and the first BM centre rows, first
+    // channel chunk), so their latency overlaps the set-up and the job table.
+    if (threadIdx.x == kWarpTma * 32) {
         for (int s = 0; s < SA; ++s) {
             mbar_init(fullA0 + 8 * s, 1);
             mbar_init(emptyA0 + 8 * s, 2);  // both issuers release every weight-ring use
@@ -247,8 +250,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(centre_done, 2);
         *abort_flag = 0;
         fence_mbar_init();
-        prefetch_tensormap(&wmap);
-        prefetch_tensormap(&xmap);
+        const int kc = p.kvol == kVol3 ? kCentre : 0;
+        mbar_arrive_expect_tx(fullA0, L::kABytes);
+        for (int box = 0; box < BM / 64; ++box)
+            tma_load_2d(smem_addr(a_ring) + box * KC * 128, &wmap, cblk * BM + box * 64, kc * p.cin, fullA0);
+        mbar_arrive_expect_tx(fullA0 + 8, L::kABytes);
+        for (int a = 0; a < L::kAtoms; ++a)
+            tma_load_2d(smem_addr(a_ring + L::kAPad) + a * BM * L::kAtomRowBytes, &xmap, a * L::kAtomElems, (int)row0,
+                        fullA0 + 8);
     }
     if (warp == kWarpMma) {
         tmem_alloc(smem_addr(tmem_slot), kTmemCols);
@@ -342,8 +351,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // centre weights then the job's BM feature rows; per offset (per job and
         // chunk when Cin spans several chunks) the offset's weights.
         if (lane == 0) {
-            int s = 0, prev_k = -1;
-            uint32_t ph = 0;
+            int s = 2 % SA, prev_k = -1;  // the first two uses were issued during set-up
+            uint32_t ph = (uint32_t)(2 / SA) & 1u;
             for (int j = 0; j < njobs && !aborted; ++j) {
                 const int4 jb = jobs[j];
                 const int k = job_k(jb);
@@ -351,6 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!centre && nchunks == 1 && k == prev_k) continue;  // same offset: the loaded tile serves
                 prev_k = k;
                 for (int c = 0; c < nchunks && !aborted; ++c) {
+                    if (j == 0 && c == 0) continue;  // issued during set-up
                     for (int part = 0; part < (centre ? 2 : 1); ++part) {
                         if (!wait_bar(emptyA0 + 8 * s, ph ^ 1u, abort_flag, p.err)) {
                             aborted = true;
