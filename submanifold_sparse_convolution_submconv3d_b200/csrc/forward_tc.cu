@@ -102,6 +102,8 @@ struct Layout {
     static constexpr int kThreadsPerRow = KC * 2 / 16;            // 16-byte chunks of one row chunk
     static constexpr int kWarpRows = 32 / kThreadsPerRow;         // rows one warp instruction covers
     static constexpr int kPasses = kJobRows / kWarpRows;
+    static constexpr int kGatherBatch = kPasses % 8 == 0 ? 8 : (kPasses % 6 == 0 ? 6 : kPasses);
+    static_assert(kPasses % kGatherBatch == 0, "gather batches must cover every pass");
     static constexpr int kChunksPerAtom = kAtomRowBytes / 16;
     static constexpr uint32_t kSwizzleMask = kAtomRowBytes / 16 - 1;
     static constexpr int kABytes = BM * KC * 2;                   // weight tile per slot
@@ -522,10 +524,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp < kWarpFold0) {
         // ------------------------------------------------ gather producers
         // Lane l copies 16-byte chunk l % kThreadsPerRow of rows
-        // l / kThreadsPerRow + kWarpRows * pass; the job's source rows are looked
-        // up once and serve every channel chunk.  Each lane arrives on the slot's
-        // barrier when its own copies land (cp.async.mbarrier.arrive.noinc), so no
-        // producer ever waits for data.
+        // l / kThreadsPerRow + kWarpRows * pass, looking the source rows up in
+        // batches.  Each lane arrives on the slot's barrier when its own copies land
+        // (cp.async.mbarrier.arrive.noinc), so no producer ever waits for data.
         const int gw = warp == 0 ? 0 : warp - 1;
         const int q = lane % L::kThreadsPerRow;
         const int prow = lane / L::kThreadsPerRow;
@@ -535,12 +536,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = ncj + gw; j < njobs && !aborted; j += kGatherWarps) {
             const int4 jb = jobs[j];
             const int n = jb.z, ncols = jb.w;
-            int src[L::kPasses];
-#pragma unroll
-            for (int ps = 0; ps < L::kPasses; ++ps) {
-                const int pr = prow + ps * L::kWarpRows;
-                src[ps] = pr < n ? pj_s[jb.y + pr] : -1;
-            }
             for (int c = 0; c < nchunks; ++c) {
                 const int slot = gw * SB + s;
                 if (!warp_wait_bar(emptyB0 + 8 * slot, ph ^ 1u, abort_flag, p.err)) {
@@ -549,14 +544,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const uint32_t b_base = smem_addr(b_ring + slot * L::kBPad) + (uint32_t)(atom * L::kBAtomBytes);
                 const __nv_bfloat16* xc = p.x + c * KC + q * 8;
+                // batches of row lookups then copies, in a rolled loop: a fully unrolled
+                // job (24 passes at 128 channels) measured 6 % slower overall
+#pragma unroll 1
+                for (int h = 0; h < L::kPasses / L::kGatherBatch; ++h) {
+                    int src[L::kGatherBatch];
 #pragma unroll
-                for (int ps = 0; ps < L::kPasses; ++ps) {
-                    const int pr = prow + ps * L::kWarpRows;
-                    if (pr < ncols) {
-                        const uint32_t lin = (uint32_t)(pr * L::kAtomRowBytes + qa * 16);
-                        const bool hit = src[ps] >= 0;
-                        cp_async_16(b_base + (lin ^ (((lin >> 7) & L::kSwizzleMask) << 4)),
-                                    xc + (int64_t)(hit ? src[ps] : 0) * p.cin, hit ? 16u : 0u);
+                    for (int i = 0; i < L::kGatherBatch; ++i) {
+                        const int pr = prow + (h * L::kGatherBatch + i) * L::kWarpRows;
+                        src[i] = pr < n ? pj_s[jb.y + pr] : -1;
+                    }
+#pragma unroll
+                    for (int i = 0; i < L::kGatherBatch; ++i) {
+                        const int pr = prow + (h * L::kGatherBatch + i) * L::kWarpRows;
+                        if (pr < ncols) {
+                            const uint32_t lin = (uint32_t)(pr * L::kAtomRowBytes + qa * 16);
+                            const bool hit = src[i] >= 0;
+                            cp_async_16(b_base + (lin ^ (((lin >> 7) & L::kSwizzleMask) << 4)),
+                                        xc + (int64_t)(hit ? src[i] : 0) * p.cin, hit ? 16u : 0u);
+                        }
                     }
                 }
                 cp_async_mbar_arrive_noinc(fullB0 + 8 * slot);
