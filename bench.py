@@ -154,6 +154,30 @@ def whole_job_mvox(world: int, steps: int, layers: int, n: int, total_ms: float)
     return world * steps * layers * n / (total_ms / 1e3) / 1e6
 
 
+def mma_column_efficiency(nbr: np.ndarray, tile_rows: int, bm: int = 128, job_rows: int = 48,
+                          n_align: int = 16) -> float:
+    """Fraction of the MMA columns the forward issues that carry a real pair.
+
+    Per tile it issues centre jobs of bm rows and, per other offset, jobs of up to
+    job_rows compacted hits; each job's MMA N is rounded up to n_align."""
+    n = nbr.shape[0]
+    t = -(-n // tile_rows)
+    hits = np.zeros((t * tile_rows, nbr.shape[1]), dtype=bool)
+    hits[:n] = nbr >= 0
+    counts = hits.reshape(t, tile_rows, -1).sum(axis=1)  # [tiles, 27]
+
+    def issued(c: np.ndarray, chunk: int) -> int:
+        rem = c % chunk
+        return int((c // chunk).sum() * chunk + ((rem + n_align - 1) // n_align * n_align).sum())
+
+    centre = nbr.shape[1] // 2
+    cols = issued(counts[:, centre], bm)
+    for k in range(nbr.shape[1]):
+        if k != centre:
+            cols += issued(counts[:, k], job_rows)
+    return float(hits.sum()) / cols
+
+
 def roofline_bytes_flops(n: int, pairs: int, cin: int, cout: int) -> tuple[float, float]:
     """Compulsory bytes and useful FLOPs of one k=3 layer: x read once, W once, bias,
     out written once, 4 bytes per non-centre neighbour pair; 2*Cin*Cout per pair."""
@@ -232,6 +256,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
 
     m = sp.spconv_build_map(coords_d, wl.grid, 3)
     pairs = m.pairs
+    col_eff = mma_column_efficiency(m.neighbor_map().cpu().numpy(), m.tile_rows)
 
     def step(events=None):
         for i in range(LAYERS):
@@ -329,7 +354,12 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         "impl": "ours",
         "layer_ms_mean": statistics.mean(layer_ms), "layer_ms_min": min(layer_ms),
         "layer_ms_median": statistics.median(layer_ms),
+        # first layer of every step: L2 was flushed just before it
+        "layer_ms_cold_l2_median": statistics.median(layer_ms[0::LAYERS]),
         "map_build_ms": statistics.median(build_ms), "pairs": pairs,
+        # build floor: coords read once + one 4-byte index per non-centre pair
+        "map_build_floor_gbs": (16 * n + 4 * (pairs - n)) / (statistics.median(build_ms) / 1e3) / 1e9,
+        "tile_rows": m.tile_rows, "mma_columns_useful_frac": col_eff,
         "roofline": {"bound": "hbm" if t_hbm >= t_tensor else "tensor", "achieved": achieved_gbs,
                      "peak": hbm, "unit": "GB/s", "frac": achieved_gbs / hbm, "traffic": traffic,
                      "traffic_source": PROFILED_TRAFFIC["profile"] if traffic is not None else None,

@@ -126,6 +126,14 @@ SPCONV_API spconv_status_t spconv_map_info(spconv_map_t map, int64_t* n, int32_t
                                 const int32_t** nbr_dev);
 
 /*
+ * Rows per tile (<= 384) that the forward kernels use with this map: chosen at
+ * build time so that the tiles fill whole waves of SMs, or forced by
+ * spconv_debug_set_tile_rows.  For reports and tests; no device work.
+ * A null `map` or `rows` returns SPCONV_ERR_INVALID_ARG.
+ */
+SPCONV_API spconv_status_t spconv_map_tile_rows(spconv_map_t map, int32_t* rows);
+
+/*
  * Synchronise `stream` and report (then clear) any device-side wait of a forward
  * kernel on this map that gave up: SPCONV_OK or SPCONV_ERR_TIMEOUT.
  */

@@ -26,6 +26,7 @@ ALGO_AUTO, ALGO_SIMT, ALGO_TCGEN05 = 0, 1, 2
 _DTYPES = {torch.float32: 0, torch.bfloat16: 1}
 
 EXPORTED = ("spconv_build_map", "spconv_subm_forward", "spconv_free", "spconv_map_info", "spconv_map_check",
+            "spconv_map_tile_rows",
             "spconv_last_error", "spconv_subm_forward_algo", "spconv_debug_set_table_slots",
             "spconv_debug_set_tile_rows", "spconv_build_neighbor_map_noalloc")
 
@@ -49,12 +50,13 @@ def _load() -> ctypes.CDLL:
     lib.spconv_map_info.argtypes = [vp, ctypes.POINTER(i64), ctypes.POINTER(i32), ctypes.POINTER(i64),
                                     ctypes.POINTER(vp)]
     lib.spconv_map_check.argtypes = [vp, vp]
+    lib.spconv_map_tile_rows.argtypes = [vp, ctypes.POINTER(i32)]
     lib.spconv_debug_set_table_slots.argtypes = [i64]
     lib.spconv_debug_set_tile_rows.argtypes = [i32]
     lib.spconv_build_neighbor_map_noalloc.argtypes = [vp, i64, vp, vp, ctypes.POINTER(i64), vp]
     lib.spconv_last_error.restype = ctypes.c_char_p
     for name in ("spconv_build_map", "spconv_subm_forward", "spconv_subm_forward_algo", "spconv_free",
-                 "spconv_map_info", "spconv_map_check", "spconv_debug_set_table_slots",
+                 "spconv_map_info", "spconv_map_check", "spconv_map_tile_rows", "spconv_debug_set_table_slots",
                  "spconv_debug_set_tile_rows", "spconv_build_neighbor_map_noalloc"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
@@ -96,6 +98,9 @@ class SubmMap:
         _check(lib.spconv_map_info(handle, ctypes.byref(n), ctypes.byref(ks), ctypes.byref(pairs), ctypes.byref(ptr)))
         self.n, self.kernel_size, self.pairs = n.value, ks.value, pairs.value
         self._nbr_ptr = ptr.value
+        rows = ctypes.c_int32()
+        _check(lib.spconv_map_tile_rows(handle, ctypes.byref(rows)))
+        self.tile_rows = rows.value  # rows per forward tile (<= 384)
 
     def neighbor_map(self) -> torch.Tensor:
         """Copy of the dense int32 [n, 27] map (identity column for kernel size 1)."""

@@ -48,6 +48,12 @@ spconv_status_t spconv_debug_set_table_slots(int64_t slots) {
     return SPCONV_OK;
 }
 
+spconv_status_t spconv_map_tile_rows(spconv_map_t map, int32_t* rows) {
+    if (!map || !rows) return fail(SPCONV_ERR_INVALID_ARG, "null map or rows");
+    *rows = map->d.tile_rows;
+    return SPCONV_OK;
+}
+
 spconv_status_t spconv_debug_set_tile_rows(int32_t rows) {
     if (rows < 0 || rows > spconv::kTileRows) return fail(SPCONV_ERR_INVALID_ARG, "rows must be in [0, 384]");
     g_tile_rows_override = rows;

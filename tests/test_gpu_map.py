@@ -94,3 +94,18 @@ def test_map_errors(sp):
         sp.spconv_debug_set_table_slots(0)
     # the library still works afterwards
     _check_map(sp, coords, (16, 16, 16))
+
+
+def test_tile_height_fills_whole_waves(sp):
+    """The map picks the smallest tile that keeps the wave count 384-row tiles need."""
+    import torch
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    wl = workloads.make_workload("uniform", 0, n_layers=1)
+    m = sp.spconv_build_map(coords_dev(wl.coords), wl.grid, 3)
+    try:
+        rows, n = m.tile_rows, wl.n
+        waves = -(-n // (384 * sms))
+        assert rows <= 384 and -(-n // rows) <= waves * sms
+        assert rows == 384 or -(-n // (rows - 1)) > waves * sms
+    finally:
+        m.free()

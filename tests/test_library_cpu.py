@@ -61,6 +61,8 @@ def test_host_validation_without_device_work(pkg):
     assert lib.spconv_subm_forward(None, 1, None, 16, None, None, None, 16, None) == pkg.INVALID_ARG
     assert lib.spconv_debug_set_table_slots(3) == pkg.INVALID_ARG
     assert lib.spconv_debug_set_table_slots(0) == pkg.OK
+    rows = ctypes.c_int32()
+    assert lib.spconv_map_tile_rows(None, ctypes.byref(rows)) == pkg.INVALID_ARG
     assert lib.spconv_debug_set_tile_rows(-1) == pkg.INVALID_ARG
     assert lib.spconv_debug_set_tile_rows(385) == pkg.INVALID_ARG
     assert lib.spconv_debug_set_tile_rows(384) == pkg.OK
