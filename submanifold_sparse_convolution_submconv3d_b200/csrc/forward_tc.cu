@@ -61,9 +61,9 @@ constexpr uint32_t kScratchCol0 = kTileRows;             // scratch buffer b at 
 constexpr uint32_t kDummyCol0 = kScratchCol0 + kScratchBufs * kJobRows;  // 480..495: fold padding targets
 static_assert(kDummyCol0 + 16 <= kTmemCols, "accumulator, scratch buffers and dummy columns must fit TMEM");
 // Warp w runs on sub-partition w % 4, and a fold warp must sit on the
-// sub-partition of its TMEM lane quarter.  The MMA issuer's sub-partition (1)
-// therefore hosts, besides three fold warps, only the light weight producer; the
-// four gather warps (0, 2, 3, 4) go to the others.
+// sub-partition of its TMEM lane quarter.  The first MMA issuer's sub-partition
+// (1) therefore hosts, besides three fold warps, only the light weight producer;
+// the four gather warps (0, 2, 3, 4) and the second issuer (18) go to the others.
 constexpr int kWarpMma = 1, kWarpTma = 5, kWarpFold0 = 6, kWarpMma2 = 18;
 constexpr int kGatherWarps = 4, kFoldWarps = 12;
 constexpr int kThreads = 32 * (kWarpFold0 + kFoldWarps + 1);  // 608
@@ -165,17 +165,14 @@ struct Params {
     int cap;  // entry capacity of the shared-memory lists (largest tile's entries)
 };
 
-// Bounded wait on an mbarrier phase.  By default the thread sleeps inside
-// try_wait; kSpin polls with test_wait instead (lowest wake-up latency, for the
-// single-thread roles on the critical path).
-template <bool kSpin = false>
+// Bounded wait on an mbarrier phase; the thread sleeps inside try_wait.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                          unsigned int* err) {
-    if (kSpin ? mbar_test_wait(bar, parity) : mbar_try_wait_hint(bar, parity, kSuspendHintNs)) return true;
+    if (mbar_try_wait_hint(bar, parity, kSuspendHintNs)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 1;; ++i) {
-        if (kSpin ? mbar_test_wait(bar, parity) : mbar_try_wait_hint(bar, parity, kSuspendHintNs)) return true;
-        if ((i & (kSpin ? 255u : 15u)) != 0) continue;  // the timer and the abort flag every few polls
+        if (mbar_try_wait_hint(bar, parity, kSuspendHintNs)) return true;
+        if ((i & 15u) != 0) continue;  // the timer and the abort flag every few wake-ups
         if (*abort_flag) return false;
         if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
             *abort_flag = 1;
