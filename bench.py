@@ -52,18 +52,24 @@ CONFIG = {
 PROFILED_TRAFFIC = {
     "kernel": "k_subm_tc<128,128>",
     "bytes": 67.150080e6 + 24.987392e6,
-    "sources_sha256": "c9fa29c75506033aec7141f1d07445be13efb786ca3a598f02d3b2d84e2e706a",
+    "sources_sha256": "763c953a69102800b323c8663025efb46b8cb6f61afb40cab3eee3bc5aac86c0",
     "profile": "profiles/k_subm_tc_uniform128.md",
 }
 KERNEL_SOURCES = ("forward_tc.cu", "sm100.cuh", "common.cuh")
 
 
 def kernel_sources_sha256() -> str:
+    """sha256 of the kernel sources' code: comments and whitespace are dropped, so
+    an edit of a comment does not retire the measured traffic, a code change does."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for name in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, "submanifold_sparse_convolution_submconv3d_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "submanifold_sparse_convolution_submconv3d_b200", "csrc", name)) as f:
+            src = f.read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", " ", src)
+        h.update(" ".join(src.split()).encode())
     return h.hexdigest()
 
 
