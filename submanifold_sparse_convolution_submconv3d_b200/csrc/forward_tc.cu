@@ -30,14 +30,16 @@
 //   warps 1, 18 TMEM allocator (warp 1) and the two tcgen05.mma issuers, which
 //               take alternate jobs
 //   warp 5      TMA producer of weight tiles (A operand), a ring of 2-6 slots
-//   warps 0, 2-4  gather producers (B operand): gather warp g fills the jobs j
-//               with j % 4 == g into its own ring of slots, in order, so each
-//               ring is filled and drained strictly in sequence
+//   warps 0, 2-4  gather producers (B operand): gather warp g fills the offset
+//               jobs ncj + q (ncj centre jobs first) with q % 4 == g into its own
+//               ring of slots, in order, so each ring is filled and drained
+//               strictly in sequence
 //   warps 6-17  scratch -> accumulator fold, then the epilogue: three warps per
 //               TMEM lane quarter, each owning the tile rows of one residue mod 3,
 //               so no accumulator column is touched by two warps of a quarter.
-//               Narrow TMEM accesses are issued without per-element branches;
-//               padding entries go to dedicated dummy columns.
+//               Narrow TMEM accesses go in batches of kNarrowGroup loads, one
+//               wait, then the stores, without per-element branches; padding
+//               entries go to dedicated dummy columns.
 // Waiting threads are suspended on their mbarrier (try_wait with a time hint)
 // and take no issue slots.  Every wait is bounded: after kWaitTimeoutNs the
 // kernel records kFwdErrTimeout in the map's error word, stops issuing work,
