@@ -77,8 +77,13 @@ typedef enum { SPCONV_F32 = 0, SPCONV_BF16 = 1 } spconv_dtype_t;
  * Device work: pack (b, x, y, z) into a 64-bit key and validate it; insert the
  * keys into an open-addressing hash table (linear probing, 64-bit CAS, load
  * factor <= 1/2); probe the 27 offsets of every voxel and write the dense map
- * nbr[i*27 + k] = row of p_i + d_k, or -1.  The call synchronises `stream`
- * once, to read the device error flags, and returns only a valid map.
+ * nbr[i*27 + k] = row of p_i + d_k, or -1.  For kernel size 3 it then builds the
+ * forward kernels' per-tile metadata: the rows are cut into tiles (height chosen
+ * for the device's SM count, see spconv_map_tile_rows), and for every tile and
+ * non-centre offset the tile rows with a neighbour there are listed.  The call
+ * synchronises `stream` twice (to read the device error flags and the metadata
+ * size, then after filling the metadata) and returns only a valid map; the hash
+ * table is freed before it returns.
  * Errors: SPCONV_ERR_COORD_RANGE, SPCONV_ERR_DUPLICATE, SPCONV_ERR_TABLE_FULL,
  * SPCONV_ERR_INVALID_ARG, SPCONV_ERR_OOM, SPCONV_ERR_CUDA.
  * The map may be used on any stream of the same device after the call returns.
@@ -100,6 +105,8 @@ SPCONV_API spconv_status_t spconv_build_map(const int32_t* coords, int64_t n, co
  *   stream  stream on which the layer runs.
  *
  * Accumulation is fp32 in every mode; the bf16 result is rounded to nearest even.
+ * bf16 with cout a multiple of 64 runs on the tensor-core (tcgen05) kernel; fp32,
+ * and bf16 with other channel counts, on a CUDA-core kernel.
  * The call only validates on the host and launches; it never synchronises.
  * Errors: SPCONV_ERR_INVALID_ARG, SPCONV_ERR_UNSUPPORTED, SPCONV_ERR_CUDA.  A
  * device-side wait that gives up is recorded in the map and reported by
