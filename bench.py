@@ -35,6 +35,11 @@ if ROOT not in sys.path:
 import workloads  # noqa: E402
 
 METRIC = "SubMConv3d Mvox/s and % of roofline at 128^3/128ch/10% occ; map-build ms"
+# The pages' own figure for this metric and workload (lato.2_mrp_mlx README, "Fleet
+# benchmark": 13.8 ms per layer on an Apple M3 Ultra, 80 GPU cores).  Another
+# machine's number: context for vs_baseline, not a target.
+PAGES_MVOX = 15.25
+PAGES_REF = "Apple M3 Ultra (80 GPU cores), 15.25 Mvox/s, lato.2_mrp_mlx README 'Fleet benchmark'; context only"
 UNIT = "Mvox/s"
 LAYERS = 10
 WORKLOAD = "uniform"
@@ -229,7 +234,8 @@ def run_reference(args, rank: int, world: int) -> None:
     base["value"] = value
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": LAYERS * wl.n / (value * 1e6) * 1e3,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": value / PAGES_MVOX, "vs_baseline_ref": PAGES_REF,
+            "dtype": "f64", "data": "synthetic",
             "config": CONFIG, "cpu_baseline": base,
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -356,7 +362,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": CONFIG,
+        "scaling": "weak", "vs_baseline": value / PAGES_MVOX, "vs_baseline_ref": PAGES_REF, "dtype": "bf16", "data": "synthetic", "config": CONFIG,
         "impl": "ours",
         "layer_ms_mean": statistics.mean(layer_ms), "layer_ms_min": min(layer_ms),
         "layer_ms_median": statistics.median(layer_ms),
