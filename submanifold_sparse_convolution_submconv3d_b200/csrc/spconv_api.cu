@@ -107,11 +107,12 @@ spconv_status_t spconv_build_map(const int32_t* coords, int64_t n, const int32_t
     int64_t entry_stats[2] = {0, 0};  // grand total, largest tile
     if (e == cudaSuccess && tiles)
         e = cudaMemcpyAsync(entry_stats, m->d.tile_off + ntiles, sizeof(entry_stats), cudaMemcpyDeviceToHost, stream);
-    const int64_t total_entries = entry_stats[0];
     if (e == cudaSuccess) e = cudaMemcpyAsync(&host_flags, flags, sizeof(host_flags), cudaMemcpyDeviceToHost, stream);
     if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
     // Second phase (only if the map is valid): entry arrays of the tile metadata.
+    // entry_stats and host_flags are read only after the synchronisation above.
     if (e == cudaSuccess && tiles && host_flags.err == 0) {
+        const int64_t total_entries = entry_stats[0];
         m->d.tile_entries = total_entries;
         m->d.tile_max_entries = entry_stats[1];
         const size_t ne = total_entries > 0 ? (size_t)total_entries : 1;
