@@ -154,15 +154,23 @@ def spconv_subm_forward(m: SubmMap, x: torch.Tensor, w: torch.Tensor, bias: torc
     for t in (w,) + (() if bias is None else (bias,)):
         if t.dtype != x.dtype or t.device != x.device:
             raise ValueError("w and bias must match x in dtype and device")
-    x, w = x.contiguous(), w.contiguous()
-    bias = None if bias is None else bias.contiguous()
+    if x.dim() != 2 or w.dim() != 3:
+        raise ValueError(f"x must be [N, Cin] and w [K^3, Cin, Cout]; got x {tuple(x.shape)}, w {tuple(w.shape)}")
     cin, cout = int(w.shape[1]), int(w.shape[2])
     if x.shape != (m.n, cin) or w.shape[0] != m.kernel_size ** 3:
         raise ValueError(f"shape mismatch: x {tuple(x.shape)}, w {tuple(w.shape)}, map n={m.n} k={m.kernel_size}")
+    if bias is not None and bias.shape != (cout,):
+        raise ValueError(f"bias must be [Cout] = [{cout}]; got {tuple(bias.shape)}")
+    if out is not None and (out.shape != (m.n, cout) or out.dtype != x.dtype or not out.is_contiguous()):
+        raise ValueError("out must be a contiguous [N, Cout] tensor of x's dtype")
+    # The library reads and writes these through raw device pointers: a host
+    # tensor, or one on another GPU than the map, must never reach it.
+    if not x.is_cuda or x.device != m.device or (out is not None and out.device != x.device):
+        raise ValueError(f"x, w, bias and out must be CUDA tensors on the map's device {m.device}")
+    x, w = x.contiguous(), w.contiguous()
+    bias = None if bias is None else bias.contiguous()
     if out is None:
         out = torch.empty((m.n, cout), dtype=x.dtype, device=x.device)
-    elif out.shape != (m.n, cout) or out.dtype != x.dtype or not out.is_contiguous():
-        raise ValueError("out must be a contiguous [N, Cout] tensor of x's dtype")
     if m.n == 0:
         return out
     with torch.cuda.device(x.device):
@@ -189,8 +197,8 @@ def spconv_build_neighbor_map_noalloc(coords: torch.Tensor, extent, out: torch.T
     n = coords.shape[0]
     if out is None:
         out = torch.empty((n, 27), dtype=torch.int32, device=coords.device)
-    elif out.shape != (n, 27) or out.dtype != torch.int32 or not out.is_contiguous():
-        raise ValueError("out must be a contiguous int32 [N, 27] tensor")
+    elif out.shape != (n, 27) or out.dtype != torch.int32 or not out.is_contiguous() or out.device != coords.device:
+        raise ValueError("out must be a contiguous int32 [N, 27] tensor on the device of coords")
     ext = (ctypes.c_int32 * 3)(*[int(v) for v in extent])
     pairs = ctypes.c_int64()
     with torch.cuda.device(coords.device):

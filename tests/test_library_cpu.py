@@ -75,3 +75,30 @@ def test_python_binding_rejects_bad_tensors(pkg):
         pkg.spconv_build_map(torch.zeros((3, 4), dtype=torch.int64), (4, 4, 4))
     with pytest.raises(ValueError):
         pkg.spconv_build_map(torch.zeros((3, 3), dtype=torch.int32), (4, 4, 4))
+
+
+def test_binding_refuses_bad_tensors_before_the_library(pkg):
+    """The binding checks shapes and devices before it passes raw pointers down:
+    a host tensor or a short bias must never reach a kernel.  The map here has no
+    library handle, so any call that got through would fail differently."""
+    import torch
+
+    m = object.__new__(pkg.SubmMap)
+    m.handle, m.device, m.n, m.kernel_size, m.pairs, m.tile_rows = None, torch.device("cuda", 0), 4, 3, 4, 4
+    x = torch.zeros((4, 16), dtype=torch.bfloat16)
+    w = torch.zeros((27, 16, 64), dtype=torch.bfloat16)
+    b = torch.zeros(64, dtype=torch.bfloat16)
+    cases = [
+        (dict(x=x, w=w, bias=b), "CUDA tensors"),                                   # host tensors
+        (dict(x=x, w=w, bias=torch.zeros(32, dtype=torch.bfloat16)), "bias must be"),  # short bias
+        (dict(x=x, w=w, bias=b.view(1, 64)), "bias must be"),
+        (dict(x=x, w=w[0]), "w [K^3, Cin, Cout]"),                                  # 2-D weights
+        (dict(x=x, w=torch.zeros((1, 16, 64), dtype=torch.bfloat16)), "shape mismatch"),
+        (dict(x=x[:3], w=w), "shape mismatch"),
+        (dict(x=x, w=w.float()), "match x"),
+        (dict(x=x, w=w, out=torch.zeros((4, 32), dtype=torch.bfloat16)), "out must be"),
+        (dict(x=x.to(torch.float16), w=w.to(torch.float16)), "float32 or bfloat16"),
+    ]
+    for kw, msg in cases:
+        with pytest.raises(ValueError, match=re.escape(msg)):
+            pkg.spconv_subm_forward(m, **kw)
