@@ -25,6 +25,11 @@
  * Conventions for every call:
  *   - Pointers documented as "device" must point to memory of the current CUDA
  *     device, 16-byte aligned.  Pointers documented as "host" are host memory.
+ *     The library checks null pointers, alignment and the documented sizes, but
+ *     it cannot tell host memory from device memory or see a buffer's length:
+ *     a host pointer, or a device buffer shorter than documented, where a device
+ *     buffer is required is undefined behaviour.  (The Python binding checks
+ *     devices and shapes before it calls in.)
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
  *     stream).
  *   - The caller owns every buffer it passes; the library keeps no pointer to a
