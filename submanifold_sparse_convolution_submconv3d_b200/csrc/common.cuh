@@ -66,9 +66,10 @@ struct MapData {
     int32_t extent[3] = {0, 0, 0};
     int64_t pairs = 0;
     int32_t* nbr = nullptr;        // device [n, 27] (kernel size 3), else null
-    // tile metadata (kernel size 3): counts [ntiles][kTileCountStride], entry offsets
-    // [ntiles + 1] (multiples of kTileEntryAlign; slot ntiles + 1 holds the largest
-    // tile's count), local rows and neighbour rows per entry
+    // tile metadata (kernel size 3): counts [ntiles][kTileCountStride]; tile_off
+    // [ntiles + 2]: each tile's first entry (multiples of kTileEntryAlign), then the
+    // grand total at slot ntiles and the largest tile's count at slot ntiles + 1;
+    // local rows and neighbour rows per entry
     int32_t* tile_counts = nullptr;
     int64_t* tile_off = nullptr;
     uint16_t* pair_r = nullptr;
