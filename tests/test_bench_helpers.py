@@ -40,3 +40,36 @@ def test_roofline_bytes_and_flops():
     byts, flops = bench.roofline_bytes_flops(n=10, pairs=30, cin=16, cout=32)
     assert byts == 10 * 16 * 2 + 27 * 16 * 32 * 2 + 32 * 2 + 10 * 32 * 2 + 4 * 20
     assert flops == 2 * 16 * 32 * 30
+
+
+def test_clock_sampler_parses_nvidia_smi_lines():
+    """Median SM clock, max clock and the throttle reasons seen, from the csv rows
+    nvidia-smi prints during the timed region (fields in ClockSampler.FIELDS order)."""
+    s = bench.ClockSampler("0")
+    s.lines = [
+        "0, 1965, 1965, 700.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "0, 1950, 1965, 980.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1965, 1965, 990.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "garbage line",
+        "0, [N/A], 1965, 1.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+    ]
+
+    class _Done:
+        def terminate(self):
+            pass
+
+        def wait(self, timeout=None):
+            return 0
+
+    s.proc = _Done()
+    c = s.stop()
+    assert c["sm_mhz"] == 1965.0 and c["sm_max_mhz"] == 1965.0 and c["samples"] == 3
+    assert c["reasons"] == ["sw_power_cap"]
+    s.lines.append("0, 1400, 1965, 990.0, 0x48, Active, Not Active, Active, Not Active")
+    c = s.stop()
+    assert c["reasons"] == ["hw_slowdown", "sw_power_cap", "sw_thermal_slowdown"]
+
+
+def test_clock_sampler_without_nvidia_smi_reports_unavailable():
+    s = bench.ClockSampler("0")
+    assert s.stop() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
