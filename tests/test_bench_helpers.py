@@ -73,3 +73,29 @@ def test_clock_sampler_parses_nvidia_smi_lines():
 def test_clock_sampler_without_nvidia_smi_reports_unavailable():
     s = bench.ClockSampler("0")
     assert s.stop() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+
+
+def test_kernel_source_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
+    """roofline.traffic is reported only while the profiled kernel's code is
+    unchanged: comment and whitespace edits keep the hash, a code edit changes it."""
+    import shutil
+
+    csrc = tmp_path / "submanifold_sparse_convolution_submconv3d_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for name in bench.KERNEL_SOURCES:
+        shutil.copy(os.path.join(ROOT, "submanifold_sparse_convolution_submconv3d_b200", "csrc", name), csrc / name)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h0 = bench.kernel_sources_sha256()
+    f = csrc / "forward_tc.cu"
+    src = f.read_text()
+    f.write_text("// a new comment line\n" + src.replace("\n", "  \n", 3) + "\n/* trailing\n block */\n")
+    assert bench.kernel_sources_sha256() == h0
+    f.write_text(src.replace("kJobRows = 48", "kJobRows = 32", 1))
+    assert bench.kernel_sources_sha256() != h0
+
+
+def test_tc_kernel_name_follows_the_dispatch():
+    assert bench.tc_kernel_name(128, 128) == "k_subm_tc<128,128>"
+    assert bench.tc_kernel_name(64, 64) == "k_subm_tc<64,64>"
+    assert bench.tc_kernel_name(48, 192) == "k_subm_tc<64,16>"
+    assert bench.tc_kernel_name(32, 256) == "k_subm_tc<128,32>"
