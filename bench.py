@@ -57,7 +57,7 @@ CONFIG = {
 PROFILED_TRAFFIC = {
     "kernel": "k_subm_tc<128,128>",
     "bytes": 67.150080e6 + 24.987392e6,
-    "sources_sha256": "763c953a69102800b323c8663025efb46b8cb6f61afb40cab3eee3bc5aac86c0",
+    "sources_sha256": "b5f00fa76987f3ceb9b3828133acef03074079d44a6779b570340136f4c31563",
     "profile": "profiles/k_subm_tc_uniform128.md",
 }
 KERNEL_SOURCES = ("forward_tc.cu", "sm100.cuh", "common.cuh")

@@ -112,6 +112,8 @@ SPCONV_API spconv_status_t spconv_build_map(const int32_t* coords, int64_t n, co
  * Accumulation is fp32 in every mode; the bf16 result is rounded to nearest even.
  * bf16 with cout a multiple of 64 runs on the tensor-core (tcgen05) kernel; fp32,
  * and bf16 with other channel counts, on a CUDA-core kernel.
+ * The layer runs on the current CUDA device, which must be the device the map
+ * was built on (otherwise SPCONV_ERR_INVALID_ARG).
  * The call only validates on the host and launches; it never synchronises.
  * Errors: SPCONV_ERR_INVALID_ARG, SPCONV_ERR_UNSUPPORTED, SPCONV_ERR_CUDA.  A
  * device-side wait that gives up is recorded in the map and reported by

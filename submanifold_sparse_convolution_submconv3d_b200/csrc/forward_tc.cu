@@ -45,6 +45,7 @@
 // kernel records kFwdErrTimeout in the map's error word, stops issuing work,
 // lets copies in flight land, frees its TMEM and returns.
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
 #include "sm100.cuh"
@@ -742,14 +743,28 @@ spconv_status_t launch(const MapData& m, const void* x, int cin, const void* w, 
         return SPCONV_ERR_CUDA;
     }
     const int smem = L::smem_bytes(cap, sa, sb);
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [&] {
-        attr_err = cudaFuncSetAttribute(k_subm_tc<BM, KC>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
-    });
-    if (attr_err != cudaSuccess) {
-        *ce = attr_err;
+    // The shared-memory opt-in is a property of the function in each device's
+    // context, so it is set once per device (and per instantiation).
+    int dev = 0;
+    cudaError_t de = cudaGetDevice(&dev);
+    if (de != cudaSuccess) {
+        *ce = de;
         return SPCONV_ERR_CUDA;
+    }
+    {
+        static std::mutex attr_mu;
+        static std::vector<char> attr_done;
+        std::lock_guard<std::mutex> lock(attr_mu);
+        if (dev >= (int)attr_done.size()) attr_done.resize((size_t)dev + 1, 0);
+        if (!attr_done[dev]) {
+            const cudaError_t ae =
+                cudaFuncSetAttribute(k_subm_tc<BM, KC>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+            if (ae != cudaSuccess) {
+                *ce = ae;
+                return SPCONV_ERR_CUDA;
+            }
+            attr_done[dev] = 1;
+        }
     }
     Params p;
     p.tile_counts = m.tile_counts;

@@ -189,6 +189,13 @@ spconv_status_t spconv_subm_forward_algo(spconv_map_t map, spconv_dtype_t dtype,
     if (dtype == SPCONV_BF16 && (cin % 16 != 0 || cout % 16 != 0))
         return fail(SPCONV_ERR_UNSUPPORTED, "bf16 needs cin and cout to be multiples of 16");
     if (map->d.n == 0) return SPCONV_OK;
+    {   // the map's buffers live on its device: launch there only
+        int dev = -1;
+        const cudaError_t de = cudaGetDevice(&dev);
+        if (de != cudaSuccess) return fail_cuda(de, "spconv_subm_forward");
+        if (dev != map->d.device)
+            return fail(SPCONV_ERR_INVALID_ARG, "the current CUDA device is not the device the map was built on");
+    }
     if (!x || !w || !out) return fail(SPCONV_ERR_INVALID_ARG, "null x, w or out");
     if (!aligned16(x) || !aligned16(w) || !aligned16(out) || (bias && !aligned16(bias)))
         return fail(SPCONV_ERR_INVALID_ARG, "x, w, bias and out must be 16-byte aligned");
