@@ -116,8 +116,10 @@ class SubmMap:
         return out
 
     def check(self, stream=None) -> None:
-        """Synchronise and raise if a forward kernel's bounded wait gave up."""
-        _check(lib.spconv_map_check(self.handle, _stream(stream)))
+        """Synchronise and raise if a forward kernel's bounded wait gave up.  The
+        default stream is the current stream of the map's device."""
+        with torch.cuda.device(self.device):
+            _check(lib.spconv_map_check(self.handle, _stream(stream)))
 
     def free(self) -> None:
         if self.handle:
