@@ -99,3 +99,18 @@ def test_tc_kernel_name_follows_the_dispatch():
     assert bench.tc_kernel_name(64, 64) == "k_subm_tc<64,64>"
     assert bench.tc_kernel_name(48, 192) == "k_subm_tc<64,16>"
     assert bench.tc_kernel_name(32, 256) == "k_subm_tc<128,32>"
+
+
+def test_column_efficiency_of_the_bench_workload():
+    """The bench reports the fraction of issued MMA columns that carry a pair. On the
+    128^3 / 10 % workload, with the 355-row tiles the library picks on 148 SMs
+    (ceil(209715 / (384 * 148)) = 4 waves, ceil(209715 / (4 * 148)) = 355 rows),
+    the oracle's map gives 85.4 %."""
+    import oracle
+    import workloads
+
+    wl = workloads.make_workload("uniform", 0, n_layers=1)
+    nbr = oracle.neighbor_map(wl.coords, wl.grid)
+    assert -(-wl.n // (384 * 148)) == 4 and -(-wl.n // (4 * 148)) == 355
+    assert int((nbr >= 0).sum()) == 745983
+    assert bench.mma_column_efficiency(nbr, 355) == pytest.approx(0.8541, abs=1e-4)
