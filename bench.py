@@ -55,12 +55,11 @@ CONFIG = {
 # (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
 # sources it was taken on: reported as null once their hash changes.
 PROFILED_TRAFFIC = {
-    "kernel": "k_subm_tc<128,128>",
-    "bytes": 67.150080e6 + 24.987392e6,
-    "sources_sha256": "b5f00fa76987f3ceb9b3828133acef03074079d44a6779b570340136f4c31563",
-    "profile": "profiles/k_subm_tc_uniform128.md",
+    "kernel": "k_subm_win<128,128>",
+    "bytes": None,
+    "sources_sha256": None,
 }
-KERNEL_SOURCES = ("forward_tc.cu", "sm100.cuh", "common.cuh")
+KERNEL_SOURCES = ("forward_win.cu", "sm100.cuh", "common.cuh")
 
 
 def kernel_sources_sha256() -> str:
@@ -82,7 +81,7 @@ def tc_kernel_name(cin: int, cout: int) -> str:
     """The forward kernel instantiation the library dispatches for these channels."""
     bm = 128 if cout % 128 == 0 else 64
     kc = 128 if cin % 128 == 0 else 64 if cin % 64 == 0 else 32 if cin % 32 == 0 else 16
-    return f"k_subm_tc<{bm},{kc}>"
+    return f"k_subm_win<{bm},{kc}>"
 
 
 def _peaks():
@@ -374,7 +373,6 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         "tile_rows": m.tile_rows, "mma_columns_useful_frac": col_eff,
         "roofline": {"bound": "hbm" if t_hbm >= t_tensor else "tensor", "achieved": achieved_gbs,
                      "peak": hbm, "unit": "GB/s", "frac": achieved_gbs / hbm, "traffic": traffic,
-                     "traffic_source": PROFILED_TRAFFIC["profile"] if traffic is not None else None,
                      "kernel": kname, "algorithmic_bytes_per_launch": byts,
                      "useful_flops_per_launch": flops, "t_hbm_us": t_hbm * 1e6, "t_tensor_us": t_tensor * 1e6,
                      "frac_of_roofline_time": max(t_hbm, t_tensor) / avg_launch_s,

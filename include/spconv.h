@@ -81,14 +81,17 @@ typedef enum { SPCONV_F32 = 0, SPCONV_BF16 = 1 } spconv_dtype_t;
  *
  * Device work: pack (b, x, y, z) into a 64-bit key and validate it; insert the
  * keys into an open-addressing hash table (linear probing, 64-bit CAS, load
- * factor <= 1/2); probe the 27 offsets of every voxel and write the dense map
- * nbr[i*27 + k] = row of p_i + d_k, or -1.  For kernel size 3 it then builds the
- * forward kernels' per-tile metadata: the rows are cut into tiles (height chosen
- * for the device's SM count, see spconv_map_tile_rows), and for every tile and
- * non-centre offset the tile rows with a neighbour there are listed.  The call
- * synchronises `stream` twice (to read the device error flags and the metadata
- * size, then after filling the metadata) and returns only a valid map; the hash
- * table is freed before it returns.
+ * factor <= 1/2); probe the 26 neighbours of every voxel and write the dense map
+ * nbr[i*27 + k] = row of p_i + d_k, or -1.  For kernel size 3 it then prepares
+ * the tensor-core forward's metadata: the rows sorted (stably, on the GPU) by the
+ * Gray-code rank of their 26-bit neighbour mask, the neighbour table in that
+ * order, and per tile of sorted rows the MMA jobs (see spconv_map_stats).
+ * Memory: every buffer comes from a stream-ordered memory pool the library keeps
+ * per device, allocated on `stream`; the hash table and sort scratch go back to
+ * the pool on `stream` before the call returns.  No cudaMalloc or cudaFree is
+ * called, and the device is not synchronised.
+ * Synchronisation: the call synchronises `stream` once, at the end, to read the
+ * device error flags, and returns only a valid map.
  * Errors: SPCONV_ERR_COORD_RANGE, SPCONV_ERR_DUPLICATE, SPCONV_ERR_TABLE_FULL,
  * SPCONV_ERR_INVALID_ARG, SPCONV_ERR_OOM, SPCONV_ERR_CUDA.
  * The map may be used on any stream of the same device after the call returns.
@@ -111,7 +114,8 @@ SPCONV_API spconv_status_t spconv_build_map(const int32_t* coords, int64_t n, co
  *
  * Accumulation is fp32 in every mode; the bf16 result is rounded to nearest even.
  * bf16 with cout a multiple of 64 runs on the tensor-core (tcgen05) kernel; fp32,
- * and bf16 with other channel counts, on a CUDA-core kernel.
+ * and bf16 with other channel counts, on a CUDA-core kernel.  The choice depends
+ * on dtype and cout alone; spconv_map_launch_counts reports which kernel ran.
  * The layer runs on the current CUDA device, which must be the device the map
  * was built on (otherwise SPCONV_ERR_INVALID_ARG).
  * The call only validates on the host and launches; it never synchronises.
@@ -123,7 +127,8 @@ SPCONV_API spconv_status_t spconv_subm_forward(spconv_map_t map, spconv_dtype_t 
                                     const void* w, const void* bias, void* out, int32_t cout,
                                     void* stream);
 
-/* Release a map and its device memory (synchronous with respect to the device).
+/* Release a map.  The call synchronises the map's device (kernels on any stream
+ * may still read the map), then returns the map's memory to the library's pool.
  * NULL is accepted and ignored. */
 SPCONV_API spconv_status_t spconv_free(spconv_map_t map);
 
@@ -140,12 +145,53 @@ SPCONV_API spconv_status_t spconv_map_info(spconv_map_t map, int64_t* n, int32_t
                                 const int32_t** nbr_dev);
 
 /*
- * Rows per tile (<= 384) that the forward kernels use with this map: chosen at
- * build time so that the tiles fill whole waves of SMs, or forced by
+ * Rows per tile (a multiple of 16, at most 256) that the tensor-core forward uses
+ * with this map: chosen at build time to even out the rows of the busiest SM when
+ * the tiles are dealt out over the device's SMs, or forced by
  * spconv_debug_set_tile_rows.  For reports and tests; no device work.
  * A null `map` or `rows` returns SPCONV_ERR_INVALID_ARG.
  */
 SPCONV_API spconv_status_t spconv_map_tile_rows(spconv_map_t map, int32_t* rows);
+
+/*
+ * The tensor-core forward's metadata of a kernel-size-3 map (for reports and
+ * tests; no device work).  The rows are sorted by the Gray-code rank of their
+ * neighbour mask (bit 25 - ks for offset k, ks = k < 13 ? k : k - 1) and cut into
+ * `tiles` tiles of `rows_per_tile` sorted rows; a tile's rows are cut into windows
+ * of 16.  For every tile and non-centre offset, the windows holding a neighbour
+ * are covered by spans of consecutive windows; each span is one tensor-core job
+ * of 16 * windows columns (holes inside it are multiplied as zero rows).
+ *   tiles, rows_per_tile  tiling of the sorted rows (0 tiles for n = 0)
+ *   spans, span_cols      spans over all tiles and the columns they cover
+ *   perm_dev              device int32 [n]: the row at each sorted position
+ *   nbr_t_dev             device int32 [27][tiles * rows_per_tile]: the neighbour
+ *                         row of sorted row r at offset k, -1 for none and for
+ *                         padding rows r >= n
+ *   jobs_dev              device uint32 [tiles][job_stride]: word 0 = job count J,
+ *                         word 1 = length of the tile's index stream (the source
+ *                         rows of all its jobs, job after job), words 2, 3 = its
+ *                         start (low, high), words 4 .. 3 + J = jobs, each k |
+ *                         first window << 8 | windows << 16; the first job is the
+ *                         centre (k = 13, all windows), the spans of each offset
+ *                         follow in increasing order
+ *   order_dev             device int32 [tiles]: the order in which the forward's
+ *                         CTAs claim the tiles, by descending estimated cost
+ *                         4 * J + stream length / 16 (stable: ties by tile index)
+ * Pointers are NULL for kernel size 1 and n = 0.  The library owns them.
+ * A null `map` or `stats` returns SPCONV_ERR_INVALID_ARG.
+ */
+typedef struct {
+    int64_t tiles;
+    int32_t rows_per_tile;
+    int32_t job_stride;
+    int64_t spans;
+    int64_t span_cols;
+    const int32_t* perm_dev;
+    const int32_t* nbr_t_dev;
+    const uint32_t* jobs_dev;
+    const int32_t* order_dev;
+} spconv_map_stats_t;
+SPCONV_API spconv_status_t spconv_map_stats(spconv_map_t map, spconv_map_stats_t* stats);
 
 /*
  * Synchronise `stream` and report (then clear) any device-side wait of a forward
@@ -171,6 +217,25 @@ SPCONV_API spconv_status_t spconv_subm_forward_algo(spconv_map_t map, spconv_dty
                                          spconv_algo_t algo, void* stream);
 
 /*
+ * Kernel families a forward can run on, for spconv_map_launch_counts.
+ */
+typedef enum {
+    SPCONV_KERNEL_SIMT = 0,     /* CUDA-core FMA kernel: fp32, and bf16 shapes no tensor-core kernel takes */
+    SPCONV_KERNEL_TCGEN05 = 1,  /* tcgen05 tensor-core kernel */
+    SPCONV_KERNEL_KINDS = 2
+} spconv_kernel_t;
+
+/*
+ * Forward launches made on this map since it was built, per kernel family:
+ * counts[k] receives the launches of family k for k < min(ncounts,
+ * SPCONV_KERNEL_KINDS); entries beyond SPCONV_KERNEL_KINDS are set to 0.  Lets a
+ * caller (and the tests) see which kernel SPCONV_ALGO_AUTO chose.  Host-side
+ * counters only: no device work.  A null map or counts, or ncounts < 1:
+ * SPCONV_ERR_INVALID_ARG.
+ */
+SPCONV_API spconv_status_t spconv_map_launch_counts(spconv_map_t map, int64_t* counts, int32_t ncounts);
+
+/*
  * Test hook: force the hash-table slot count of later builds in this process
  * (0 restores the automatic choice, a power of two >= 2n).  Lets a test reach
  * SPCONV_ERR_TABLE_FULL with a small table.  `slots` must be 0 or a power of two.
@@ -178,13 +243,22 @@ SPCONV_API spconv_status_t spconv_subm_forward_algo(spconv_map_t map, spconv_dty
 SPCONV_API spconv_status_t spconv_debug_set_table_slots(int64_t slots);
 
 /*
- * Test hook: force the tile height (rows per forward CTA, 1..384) of later builds
- * in this process; 0 restores the automatic choice, the smallest height that
- * fills the same number of waves of SMs as 384-row tiles.  Lets tests run small
- * inputs through full-height tiles (several jobs per offset).  Other values:
- * SPCONV_ERR_INVALID_ARG.
+ * Test hook: force the tile height (sorted rows per tile, a multiple of 16 in
+ * [16, 256]) of later builds in this process; 0 restores the automatic choice.
+ * Lets tests run small inputs through full-height tiles and many short tiles.
+ * Other values: SPCONV_ERR_INVALID_ARG.
  */
 SPCONV_API spconv_status_t spconv_debug_set_tile_rows(int32_t rows);
+
+/*
+ * Test hook: force the tensor-core forward's ring depths for later launches in
+ * this process: a_slots weight tiles in [2, 8] and b_units units of 64 gathered
+ * rows in [4, 32]; (0, 0) restores the automatic choice.  A launch whose forced
+ * depths do not fit shared memory returns SPCONV_ERR_UNSUPPORTED.  Lets tests
+ * drive shallow rings (frequent wrap-around) and the benchmark sweep depths.
+ * Other values: SPCONV_ERR_INVALID_ARG.
+ */
+SPCONV_API spconv_status_t spconv_debug_set_ring_depths(int32_t a_slots, int32_t b_units);
 
 /*
  * Neighbour-map build that allocates no device memory.  The pages have no
@@ -205,11 +279,15 @@ SPCONV_API spconv_status_t spconv_debug_set_tile_rows(int32_t rows);
  *
  * The hash table and error flags live in one static device array of 16 MiB plus
  * 256 bytes that every GPU loading this library holds until the process exits.
- * The first call on a device looks up that array's device address (with the
- * device current); make that first call before any stream capture.  Every call
- * shares the array and clears it before use, so calls that overlap on the GPU
- * (on different streams or host threads) race and must not be issued.  Errors:
- * as spconv_build_map, plus SPCONV_ERR_UNSUPPORTED above the size limit;
+ * Every call looks up that array's device address with the calling thread's
+ * current device (the lookup allocates nothing), so the entry point stays valid
+ * after a device reset.  The first call on a device may load the library's
+ * device code there.  Every call shares the array and clears it before use, so
+ * calls that overlap on the GPU (on different streams or host threads) race and
+ * must not be issued.  The call copies the error flags to host memory and
+ * synchronises `stream` before it returns, so it must never be issued while
+ * `stream` (or any stream it would join) is being captured into a CUDA graph.
+ * Errors: as spconv_build_map, plus SPCONV_ERR_UNSUPPORTED above the size limit;
  * spconv_last_error() describes them.
  */
 SPCONV_API spconv_status_t spconv_build_neighbor_map_noalloc(const int32_t* coords, int64_t n, const int32_t* extent,

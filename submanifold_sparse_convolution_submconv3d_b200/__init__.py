@@ -23,12 +23,21 @@ LIB_PATH = os.path.join(_HERE, "libspconv_b200.so")
 
 OK, INVALID_ARG, UNSUPPORTED, COORD_RANGE, DUPLICATE, TABLE_FULL, OOM, CUDA_ERROR, TIMEOUT = range(9)
 ALGO_AUTO, ALGO_SIMT, ALGO_TCGEN05 = 0, 1, 2
+KERNEL_SIMT, KERNEL_TCGEN05 = 0, 1
+KERNEL_NAMES = ("simt", "tcgen05")
 _DTYPES = {torch.float32: 0, torch.bfloat16: 1}
 
 EXPORTED = ("spconv_build_map", "spconv_subm_forward", "spconv_free", "spconv_map_info", "spconv_map_check",
             "spconv_map_tile_rows",
             "spconv_last_error", "spconv_subm_forward_algo", "spconv_debug_set_table_slots",
-            "spconv_debug_set_tile_rows", "spconv_build_neighbor_map_noalloc")
+            "spconv_debug_set_tile_rows", "spconv_build_neighbor_map_noalloc", "spconv_map_launch_counts",
+            "spconv_map_stats", "spconv_debug_set_ring_depths")
+
+
+class _MapStats(ctypes.Structure):
+    _fields_ = [("tiles", ctypes.c_int64), ("rows_per_tile", ctypes.c_int32), ("job_stride", ctypes.c_int32),
+                ("spans", ctypes.c_int64), ("span_cols", ctypes.c_int64), ("perm_dev", ctypes.c_void_p),
+                ("nbr_t_dev", ctypes.c_void_p), ("jobs_dev", ctypes.c_void_p), ("order_dev", ctypes.c_void_p)]
 
 
 class SpconvError(RuntimeError):
@@ -54,10 +63,14 @@ def _load() -> ctypes.CDLL:
     lib.spconv_debug_set_table_slots.argtypes = [i64]
     lib.spconv_debug_set_tile_rows.argtypes = [i32]
     lib.spconv_build_neighbor_map_noalloc.argtypes = [vp, i64, vp, vp, ctypes.POINTER(i64), vp]
+    lib.spconv_map_launch_counts.argtypes = [vp, ctypes.POINTER(i64), i32]
+    lib.spconv_map_stats.argtypes = [vp, ctypes.POINTER(_MapStats)]
+    lib.spconv_debug_set_ring_depths.argtypes = [i32, i32]
     lib.spconv_last_error.restype = ctypes.c_char_p
     for name in ("spconv_build_map", "spconv_subm_forward", "spconv_subm_forward_algo", "spconv_free",
                  "spconv_map_info", "spconv_map_check", "spconv_map_tile_rows", "spconv_debug_set_table_slots",
-                 "spconv_debug_set_tile_rows", "spconv_build_neighbor_map_noalloc"):
+                 "spconv_debug_set_tile_rows", "spconv_build_neighbor_map_noalloc", "spconv_map_launch_counts",
+                 "spconv_map_stats", "spconv_debug_set_ring_depths"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -102,18 +115,43 @@ class SubmMap:
         _check(lib.spconv_map_tile_rows(handle, ctypes.byref(rows)))
         self.tile_rows = rows.value  # rows per forward tile (<= 384)
 
+    def _copy_device(self, ptr: int, shape: tuple, typestr: str, dtype) -> torch.Tensor:
+        """Copy of a library-owned device buffer, viewed through the CUDA array interface."""
+        out = torch.empty(shape, dtype=dtype, device=self.device)
+        if out.numel():
+            class _View:
+                __cuda_array_interface__ = {"shape": shape, "typestr": typestr, "data": (ptr, False), "version": 3}
+            out.copy_(torch.as_tensor(_View(), device=self.device))
+        return out
+
     def neighbor_map(self) -> torch.Tensor:
         """Copy of the dense int32 [n, 27] map (identity column for kernel size 1)."""
         if self.kernel_size == 1:
             return torch.arange(self.n, dtype=torch.int32, device=self.device).view(-1, 1)
-        out = torch.empty((self.n, 27), dtype=torch.int32, device=self.device)
-        if self.n:
-            # View the library-owned buffer through the CUDA array interface and copy it.
-            class _View:
-                __cuda_array_interface__ = {"shape": (self.n, 27), "typestr": "<i4",
-                                            "data": (self._nbr_ptr, False), "version": 3}
-            out.copy_(torch.as_tensor(_View(), device=self.device))
-        return out
+        return self._copy_device(self._nbr_ptr, (self.n, 27), "<i4", torch.int32)
+
+    def stats(self, copy_arrays: bool = False) -> dict:
+        """The tensor-core forward's metadata (spconv_map_stats): tiling, span counts
+        and, with copy_arrays, copies of perm [n], nbr_t [27, tiles * rows_per_tile],
+        jobs [tiles, job_stride] (uint32 words as int64) and order [tiles]."""
+        st = _MapStats()
+        _check(lib.spconv_map_stats(self.handle, ctypes.byref(st)))
+        d = {"tiles": st.tiles, "rows_per_tile": st.rows_per_tile, "job_stride": st.job_stride, "spans": st.spans,
+             "span_cols": st.span_cols}
+        if copy_arrays and st.perm_dev:
+            npad = st.tiles * st.rows_per_tile
+            d["perm"] = self._copy_device(st.perm_dev, (self.n,), "<i4", torch.int32)
+            d["nbr_t"] = self._copy_device(st.nbr_t_dev, (27, npad), "<i4", torch.int32)
+            d["jobs"] = self._copy_device(st.jobs_dev, (st.tiles, st.job_stride), "<i4",
+                                          torch.int32).to(torch.int64) & 0xFFFFFFFF
+            d["order"] = self._copy_device(st.order_dev, (st.tiles,), "<i4", torch.int32)
+        return d
+
+    def launch_counts(self) -> dict:
+        """Forward launches on this map per kernel family, e.g. {"simt": 0, "tcgen05": 3}."""
+        counts = (ctypes.c_int64 * len(KERNEL_NAMES))()
+        _check(lib.spconv_map_launch_counts(self.handle, counts, len(KERNEL_NAMES)))
+        return dict(zip(KERNEL_NAMES, counts))
 
     def check(self, stream=None) -> None:
         """Synchronise and raise if a forward kernel's bounded wait gave up.  The
@@ -220,8 +258,14 @@ def spconv_debug_set_tile_rows(rows: int) -> None:
     _check(lib.spconv_debug_set_tile_rows(int(rows)))
 
 
+def spconv_debug_set_ring_depths(a_slots: int, b_units: int) -> None:
+    _require()
+    _check(lib.spconv_debug_set_ring_depths(int(a_slots), int(b_units)))
+
+
 __all__ = ["OK", "INVALID_ARG", "UNSUPPORTED", "COORD_RANGE", "DUPLICATE", "TABLE_FULL", "OOM", "CUDA_ERROR",
            "TIMEOUT", "SubmMap", "SpconvError", "spconv_build_map", "spconv_subm_forward", "spconv_free",
-           "spconv_debug_set_table_slots", "spconv_debug_set_tile_rows", "spconv_build_neighbor_map_noalloc", "lib",
+           "spconv_debug_set_table_slots", "spconv_debug_set_tile_rows", "spconv_debug_set_ring_depths",
+           "spconv_build_neighbor_map_noalloc", "lib",
            "LIB_PATH", "EXPORTED",
-           "ALGO_AUTO", "ALGO_SIMT", "ALGO_TCGEN05"]
+           "ALGO_AUTO", "ALGO_SIMT", "ALGO_TCGEN05", "KERNEL_SIMT", "KERNEL_TCGEN05", "KERNEL_NAMES"]

@@ -16,6 +16,7 @@ enum : unsigned int {
     kErrCoordRange = 1u,
     kErrDuplicate = 2u,
     kErrTableFull = 4u,
+    kErrInternal = 8u,  // a bound the metadata relies on did not hold (not expected)
 };
 
 // Device-side error bits written by forward kernels into the map's error word.
@@ -26,37 +27,59 @@ enum : unsigned int {
 struct BuildFlags {
     unsigned int err;
     unsigned int pad;
-    unsigned long long pairs;  // (voxel, offset) pairs with an active neighbour, centre included
+    unsigned long long pairs;      // (voxel, offset) pairs with an active neighbour, centre included
+    unsigned long long spans;      // window-kernel spans over all tiles
+    unsigned long long span_cols;  // columns those spans cover
+    unsigned long long max_tile_cols;  // longest per-tile index stream (columns of all its jobs)
 };
 
 // Offset order used everywhere: k = (dx+1)*9 + (dy+1)*3 + (dz+1).
 constexpr int kVol3 = 27;
 constexpr int kCentre = 13;
 
-// Tile metadata (built with the map, kernel size 3): the rows are cut into tiles
-// of `tile_rows` consecutive rows (at most kTileRows, chosen per map by
-// choose_tile_rows); for every tile and every non-centre offset the
-// tile rows with an active neighbour there are listed, split into three classes
-// by row % 3 and sorted by row within a class.  "Units" are (offset, class)
-// pairs in offset-major order, offsets 0..26 without the centre: unit
-// u = 3 * ks + c with ks = k < 13 ? k : k - 1.
-constexpr int kTileRows = 384;
-constexpr int kTileClasses = 3;
-constexpr int kTileUnits = (kVol3 - 1) * kTileClasses;  // 78
-constexpr int kTileCountStride = 80;                    // int32 counts per tile (78 used), 320 bytes
-constexpr int kTileEntryAlign = 8;                      // each tile's entries start on a multiple of 8
+// Window-kernel metadata (kernel size 3).  The rows are reordered by their
+// neighbour pattern: the 26 non-centre hit bits of a row form a mask, and the rows
+// are sorted (stably) by the rank of that mask in the reflected Gray-code order,
+// so rows with similar patterns sit next to each other and each offset's hits
+// bunch into runs.  The sorted rows are cut into tiles of win_rows rows (a
+// multiple of kWinCols, at most kWinMaxRows) and each tile into windows of
+// kWinCols rows.  For every tile and non-centre offset, the windows holding a hit
+// are covered by spans of consecutive windows (chosen by a cost model of the MMA,
+// see map_window.cu); one span is one MMA of N = 16 * windows columns.  A tile's
+// job list is its centre job (every row, N = win_rows) followed by its spans.
+constexpr int kWinCols = 16;                 // rows per window (MMA N granule)
+constexpr int kWinMaxRows = 256;             // rows per tile at most (one TMEM accumulator)
+constexpr int kWinMaxSpans = 8;              // spans per (tile, offset) at most: kWinMaxRows / kWinCols / 2
+// A tile's record (uint32 words): [0] job count J, [1] index-stream entries,
+// [2], [3] index-stream start (low, high word), then J job words (the centre job
+// first), padded to kWinJobStride words (a multiple of 4, so records stay 16-byte
+// aligned for bulk copies).
+constexpr int kWinRecHeader = 4;
+constexpr int kWinJobStride = 216;           // header + centre job + <= 26 * 8 spans, padding
+// Job word: offset k in bits 0-4, first window in bits 8-12, window count in bits 16-20.
+__host__ __device__ inline uint32_t win_job(int k, int w0, int nw) {
+    return (uint32_t)k | ((uint32_t)w0 << 8) | ((uint32_t)nw << 16);
+}
+__host__ __device__ inline int win_job_k(uint32_t j) { return (int)(j & 31u); }
+__host__ __device__ inline int win_job_w0(uint32_t j) { return (int)((j >> 8) & 31u); }
+__host__ __device__ inline int win_job_nw(uint32_t j) { return (int)((j >> 16) & 31u); }
 
-__host__ __device__ inline int64_t num_tiles(int64_t n, int tile_rows) { return (n + tile_rows - 1) / tile_rows; }
-
-// Rows per tile for n voxels on num_sms SMs (one tile per SM at a time): the
-// number of waves that kTileRows-row tiles need, then the smallest tile that
-// still fits n into that many waves, so the last wave is not left mostly empty.
-inline int choose_tile_rows(int64_t n, int num_sms) {
-    if (n <= 0 || num_sms <= 0) return kTileRows;
-    const int64_t per_wave = (int64_t)kTileRows * num_sms;
-    const int64_t waves = (n + per_wave - 1) / per_wave;
-    const int64_t rows = (n + waves * num_sms - 1) / (waves * num_sms);
-    return (int)(rows < 32 ? (n < 32 ? n : 32) : rows);
+// Window-tile height for n rows on num_sms SMs: the multiple of kWinCols in
+// [128, kWinMaxRows] that minimises the rows of the busiest SM when tiles are
+// dealt out round-robin (ties: the taller tile).
+inline int choose_win_rows(int64_t n, int num_sms) {
+    if (n <= 0 || num_sms <= 0) return kWinMaxRows;
+    int best = kWinMaxRows;
+    int64_t best_load = -1;
+    for (int r = kWinMaxRows; r >= 128; r -= kWinCols) {
+        const int64_t tiles = (n + r - 1) / r;
+        const int64_t load = (tiles + num_sms - 1) / num_sms * r;
+        if (best_load < 0 || load < best_load) {
+            best_load = load;
+            best = r;
+        }
+    }
+    return best;
 }
 
 // The map handle (defined here so the launchers can read it).
@@ -66,39 +89,65 @@ struct MapData {
     int32_t extent[3] = {0, 0, 0};
     int64_t pairs = 0;
     int32_t* nbr = nullptr;        // device [n, 27] (kernel size 3), else null
-    // tile metadata (kernel size 3): counts [ntiles][kTileCountStride]; tile_off
-    // [ntiles + 2]: each tile's first entry (multiples of kTileEntryAlign), then the
-    // grand total at slot ntiles and the largest tile's count at slot ntiles + 1;
-    // local rows and neighbour rows per entry
-    int32_t* tile_counts = nullptr;
-    int64_t* tile_off = nullptr;
-    uint16_t* pair_r = nullptr;
-    int32_t* pair_j = nullptr;
-    int64_t tile_entries = 0;
-    int64_t tile_max_entries = 0;  // entries of the fullest tile (a multiple of kTileEntryAlign)
-    int32_t tile_rows = kTileRows;  // rows per tile (<= kTileRows), for the forward kernels too
+    // window-kernel metadata (kernel size 3): perm [n] (sorted position -> row);
+    // nbr_t [27][npad], the neighbour row of sorted row r at offset k or -1 (rows
+    // r >= n are padding, all -1); win_jobs [win_tiles][kWinJobStride]
+    int32_t* perm = nullptr;
+    int32_t* nbr_t = nullptr;
+    uint32_t* win_jobs = nullptr;
+    int64_t npad = 0;
+    int64_t win_tiles = 0;
+    int32_t win_rows = kWinMaxRows;
+    // per-tile index streams: the source rows of every job of the tile, job after
+    // job; tile t's stream is idx_stream[idx_off[t] .. idx_off[t + 1])
+    int32_t* idx_stream = nullptr;
+    int64_t* idx_off = nullptr;
+    int64_t max_tile_cols = 0;
+    // work counters of the forward's tile scheduler: a launch takes slot
+    // (launch number % kSchedSlots), cleared on its stream just before it
+    uint32_t* sched = nullptr;
+    int32_t* win_order = nullptr;  // [win_tiles] tiles in claim order (most expensive first)
+    int64_t win_spans = 0;         // spans over all tiles (MMA jobs besides the centre)
+    int64_t win_span_cols = 0;     // columns those spans cover
     unsigned int* fwd_err = nullptr;  // device word: forward-kernel error bits
     int device = 0;
     int num_sms = 0;
 };
 
+constexpr int kSchedSlots = 64;
+
 // Sets the calling thread's message returned by spconv_last_error().
 void set_last_error(const std::string& msg);
 
 // Launchers (each returns cudaSuccess or the first CUDA error).
+// Pack + validate + insert, then (kernel size 3) probe into the dense map `nbr`
+// and, when `keys` is not null, the rows' sort keys (Gray rank of the neighbour mask).
 cudaError_t launch_build_map(const int32_t* coords, int64_t n, const int32_t extent[3], int32_t kernel_size,
-                             unsigned long long* table, uint64_t slots, int32_t* nbr, BuildFlags* flags,
-                             cudaStream_t stream);
+                             unsigned long long* table, uint64_t slots, int32_t* nbr, uint32_t* keys,
+                             BuildFlags* flags, cudaStream_t stream);
 
-// Tile metadata in two passes: counts + offsets (then the caller reads the total
-// and allocates the entry arrays), then the entries.
-cudaError_t launch_tile_count(const int32_t* nbr, int64_t n, int tile_rows, int32_t* tile_counts, int64_t* tile_off,
-                              cudaStream_t stream);
-cudaError_t launch_tile_fill(const int32_t* nbr, int64_t n, int tile_rows, const int32_t* tile_counts,
-                             const int64_t* tile_off, uint16_t* pair_r, int32_t* pair_j, cudaStream_t stream);
+// Stable radix sort of (key, value) pairs by the low key_bits bits: keys[0] holds
+// the input keys and vals_in the input values (null: the element indices);
+// keys[1], vals[0] and vals[1] are buffers of n elements; hist holds
+// radix_hist_words(n) words.  The sorted pairs end in keys[*which], vals[*which].
+int64_t radix_hist_words(int64_t n);
+cudaError_t radix_sort_pairs(uint32_t* keys[2], const int32_t* vals_in, int32_t* vals[2], int64_t n, int key_bits,
+                             uint32_t* hist, int* which, cudaStream_t stream);
+
+// Window-kernel metadata from the dense map and the sorted rows.
+cudaError_t launch_win_meta(const int32_t* nbr, const int32_t* sorted_rows, int64_t n, int rows, int64_t tiles,
+                            int64_t npad, int32_t* perm, int32_t* nbr_t, uint32_t* jobs, int64_t* idx_off,
+                            int32_t* idx_stream, BuildFlags* flags, cudaStream_t stream);
+
+// Sort keys of the tile claim order (ascending key = descending estimated cost).
+cudaError_t launch_win_cost(const uint32_t* jobs, int64_t tiles, uint32_t* keys, cudaStream_t stream);
 
 cudaError_t launch_forward_simt(const MapData& m, spconv_dtype_t dtype, const void* x, int cin, const void* w,
                                 const void* bias, void* out, int cout, cudaStream_t stream);
+
+// Test hook of the tensor-core forward: force the weight-ring slots and B-ring
+// units of later launches (0, 0: automatic).
+void set_forced_ring_depths(int sa, int ub);
 
 // Returns SPCONV_OK, SPCONV_ERR_UNSUPPORTED (shape not handled) or SPCONV_ERR_CUDA.
 spconv_status_t launch_forward_tcgen05(const MapData& m, const void* x, int cin, const void* w,

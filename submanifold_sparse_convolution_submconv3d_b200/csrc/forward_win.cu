@@ -1,0 +1,778 @@
+// Fused gather -> tcgen05 GEMM -> single-write store over sorted windows.
+//
+// The pages fuse the 27 per-offset taps into one [N, 27*Cin] x [27*Cin, Cout]
+// matmul over a cached device index (lato.2_mrp_mlx README, "Fleet benchmark"
+// and the optimisation table after it).  This kernel computes the same sum,
+//
+//   D^T[Cout_blk, rows] = sum_k W_k^T[Cout_blk, Cin] . X_k^T[Cin, rows],
+//
+// laid out for sm_100a.  The map build has sorted the rows by neighbour pattern
+// and recorded, per tile of consecutive sorted rows, the jobs: the centre job (all
+// rows of the tile) and, per non-centre offset, spans of consecutive 16-row
+// windows holding its hits, plus one contiguous stream of the jobs' source rows
+// (map_window.cu).  A job is one run of MMAs whose output columns are the tile's
+// own accumulator columns, so every product lands in place: no scatter, no fold,
+// no atomics.  Holes inside a span are gathered as zero rows.
+//
+// Persistent CTAs (one per SM) take (tile, output-channel block) units from a
+// work counter, so CTAs that drew cheap tiles take more of them.  Tensor memory
+// holds two accumulators of 256 columns (lane = output channel, column = sorted
+// row of the tile), so the epilogue of one tile overlaps the MMAs of the next.
+//
+// Warp roles (448 threads):
+//   warp 0      TMEM allocator; lane 0 issues every tcgen05.mma and commit
+//   warp 1      lane 0: claims units (tiles in the map's claim order, most
+//               expensive first) and copies each unit's tile record (job list and
+//               index-stream position) into a ring of four shared-memory slots,
+//               two units ahead; then, as TMA producer, loads the weight
+//               tiles W_k (A operand, MN-major straight from the [K^3 * Cin, Cout]
+//               weights) into a ring of slots
+//   warps 2-5   gather producers (B operand).  A tile's index stream arrives in
+//               shared memory by one bulk copy, a tile ahead, into one of two
+//               buffers.  The B ring is cut into units of 64 rows; a job takes
+//               ceil(N / 64) consecutive units (never wrapping); all four warps
+//               fill every unit, 16 rows each, with 16-byte cp.async copies (zero
+//               fill for holes) into the swizzled K-major layout the MMA reads, so
+//               each unit's uses are filled and drained strictly in turn
+//   warps 6-13  epilogue: two warps per TMEM lane quarter, alternate 32-column
+//               chunks: accumulator + bias -> bf16, staged in shared memory, then
+//               16-byte stores to each output row, written exactly once; output
+//               rows and bias are fetched before the accumulator is ready
+// Every wait is bounded: after kWaitTimeoutNs the kernel records kFwdErrTimeout
+// in the map's error word, stops issuing work, lets copies in flight land, waits
+// (bounded) for its MMAs and frees its TMEM before returning.
+#include <atomic>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace spconv {
+namespace {
+
+using namespace sm100;
+
+constexpr int kWarpMma = 0, kWarpTma = 1, kWarpGather0 = 2, kGatherWarps = 4, kWarpEpi0 = 6, kEpiWarps = 8;
+constexpr int kThreads = 32 * (kWarpEpi0 + kEpiWarps);  // 448
+constexpr int kAccBufs = 2;
+constexpr int kIdxBufs = 2;
+constexpr int kTileSlots = 4;          // tile-record ring
+constexpr int kTileConsumers = 1 + kGatherWarps + kEpiWarps;  // arrivals that free a tile slot
+constexpr int kRecBytes = kWinJobStride * 4;
+constexpr int kSlotBytes = 16 + kRecBytes;  // [unit id][pad][record]
+static_assert(kRecBytes % 16 == 0 && kSlotBytes % 16 == 0, "tile records are bulk-copied");
+constexpr uint32_t kAccCols = kWinMaxRows;  // 256 columns per accumulator
+constexpr uint32_t kTmemCols = 512;
+static_assert(kAccBufs * kAccCols <= kTmemCols, "accumulators must fit TMEM");
+constexpr int kUnitRows = 64;          // rows of one B-ring unit
+constexpr int kMaxUnits = 32;          // the per-unit phase bits live in one 32-bit word
+constexpr int kMaxASlots = 8;
+constexpr uint64_t kWaitTimeoutNs = 4000000000ull;
+constexpr int kMaxSmem = 232448;       // 227 KB opt-in limit per CTA on sm_100
+constexpr int kMinSmem = 120 * 1024;   // keeps one CTA per SM: each CTA allocates all 512 TMEM columns
+
+__host__ __device__ constexpr int round_up(int v, int m) { return (v + m - 1) / m * m; }
+
+template <int BM, int KC>
+struct WinLayout {
+    // B: gathered rows, K-major, split into swizzle atoms of up to 64 channels
+    // (128 bytes); ring layout [atom][unit][64 rows][atom row bytes], so the rows
+    // of consecutive units are contiguous for the MMA descriptor.
+    static constexpr int kAtomElems = KC >= 64 ? 64 : KC;
+    static constexpr int kAtoms = KC / kAtomElems;
+    static constexpr int kARB = kAtomElems * 2;                // atom row bytes: 128, 64 or 32
+    static constexpr int kUnitAtomBytes = kUnitRows * kARB;    // a multiple of the swizzle repeat
+    static constexpr int kUnitBytes = kAtoms * kUnitAtomBytes;
+    static constexpr int kThreadsPerRow = KC * 2 / 16;         // 16-byte chunks of one row's chunk
+    static constexpr int kWarpRows = 32 / kThreadsPerRow;      // rows one warp instruction covers
+    static constexpr int kSliceRows = kUnitRows / kGatherWarps;  // rows of a unit one gather warp fills
+    static constexpr int kPasses = kSliceRows / kWarpRows;
+    static_assert(kPasses >= 1 && kSliceRows % kWarpRows == 0, "a slice must split into whole passes");
+    static constexpr int kChunksPerAtom = kARB / 16;
+    static constexpr uint32_t kSwz = kARB / 16 - 1;
+    static constexpr uint32_t kBLayout = kARB == 128 ? 2u : (kARB == 64 ? 4u : 6u);
+    static constexpr uint32_t kBSbo = 8 * kARB;
+    static constexpr int kStepsPerAtom = kAtomElems / 16;
+    // A: weights, MN-major, BM / 64 boxes of [KC rows][64 channels], 128-byte swizzle.
+    static constexpr int kABytes = BM * KC * 2;
+    static constexpr int kAPad = round_up(kABytes, 1024);
+    static constexpr int kChPerWarp = BM / 4;  // output channels of one TMEM lane quarter
+    static constexpr int kStageRows = 16;      // output rows one epilogue warp stages at a time
+    static constexpr int kStageBytes = kEpiWarps * kStageRows * kChPerWarp * 2;
+
+    // A tile's index buffer: its stream plus one unit of slack (the last unit of a
+    // job may read past the job's columns; those reads are masked).
+    __host__ __device__ static int idx_buf_bytes(int max_cols) { return round_up((max_cols + kUnitRows) * 4, 128); }
+    __host__ __device__ static int ring_bytes(int sa, int ub) { return sa * kAPad + ub * kUnitBytes; }
+    __host__ __device__ static int num_bars(int sa, int ub) {
+        return 2 * sa + 2 * ub + 2 * kAccBufs + 2 * kIdxBufs + 2 * kTileSlots + 1;
+    }
+    __host__ __device__ static int smem_bytes(int sa, int ub, int max_cols) {
+        return 1024 + ring_bytes(sa, ub) + kStageBytes + kIdxBufs * idx_buf_bytes(max_cols) +
+               kTileSlots * kSlotBytes + num_bars(sa, ub) * 8 + 16;
+    }
+};
+
+struct WinParams {
+    const int32_t* perm;        // [n] sorted row -> row (null: identity, kernel size 1)
+    const uint32_t* recs;       // [tiles][kWinJobStride] tile records (null for kernel size 1)
+    const int32_t* idx_stream;  // per-tile source rows of every job (null for kernel size 1)
+    const int32_t* order;       // [tiles] claim order of the tiles (null: natural order)
+    unsigned int* work;         // this launch's work counter, zero at launch
+    int64_t n, tiles;
+    int rows;                   // rows per tile (multiple of 16, <= 256)
+    int cblocks;                // output-channel blocks of BM
+    const __nv_bfloat16* x;
+    int cin;
+    const __nv_bfloat16* bias;
+    __nv_bfloat16* out;
+    int cout;
+    unsigned int* err;
+    int sa, ub;                 // weight-ring slots, B-ring units
+    int idx_buf_elems;          // int32 entries of one tile index buffer
+};
+
+// Waiting policy.  A waiting thread polls the barrier; while the phase is not
+// complete it backs off with __nanosleep, doubling the pause up to its role's
+// ceiling, so waiting warps leave the issue slots to the warps doing work.  The
+// MMA issuer waits on data that is usually about to land and does not pause;
+// producers wait for ring slots; the epilogue waits for a whole tile of MMAs.
+constexpr uint32_t kSleepMma = 0, kSleepProducer = 128, kSleepEpilogue = 2048;
+
+template <uint32_t kMaxSleepNs>
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag, unsigned int* err) {
+    if (mbar_try_wait(bar, parity)) return true;
+    uint64_t t0 = 0;
+    uint32_t pause = 32;
+    for (uint32_t i = 1;; ++i) {
+        if constexpr (kMaxSleepNs > 0) {
+            __nanosleep(pause);
+            pause = pause < kMaxSleepNs ? 2 * pause : pause;
+        }
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 15u) != 0) continue;  // the timer and the abort flag every few polls
+        if (*abort_flag) return false;
+        const uint64_t now = globaltimer_ns();
+        if (t0 == 0) {
+            t0 = now;
+        } else if (now - t0 > kWaitTimeoutNs) {
+            *abort_flag = 1;
+            atomicOr(err, kFwdErrTimeout);
+            return false;
+        }
+    }
+}
+
+template <uint32_t kMaxSleepNs>
+__device__ __forceinline__ bool warp_wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                              unsigned int* err) {
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0) ok = wait_bar<kMaxSleepNs>(bar, parity, abort_flag, err) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// B-ring units of the next (job, chunk): ceil(N / 64) consecutive units, starting
+// over at unit 0 when they would run past the end.  Every role runs this on the
+// same sequence, so all agree on the placement.
+__device__ __forceinline__ int alloc_units(int& ucur, int ub, int ncols, int* m) {
+    *m = (ncols + kUnitRows - 1) / kUnitRows;
+    if (ucur + *m > ub) ucur = 0;
+    const int u0 = ucur;
+    ucur += *m;
+    return u0;
+}
+
+// A tile slot: word 0 the claimed tile (-1: no more work), word 1 its output-channel
+// block, words 4.. the tile's record.
+__device__ __forceinline__ int slot_unit(const uint8_t* slot) { return *reinterpret_cast<const volatile int*>(slot); }
+__device__ __forceinline__ int slot_cblk(const uint8_t* slot) {
+    return *reinterpret_cast<const volatile int*>(slot + 4);
+}
+__device__ __forceinline__ const uint32_t* slot_rec(const uint8_t* slot) {
+    return reinterpret_cast<const uint32_t*>(slot + 16);
+}
+
+template <int BM, int KC>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_subm_win(const __grid_constant__ CUtensorMap wmap, const WinParams p) {
+    using L = WinLayout<BM, KC>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int SA = p.sa, UB = p.ub;
+    uint8_t* a_ring = smem;
+    uint8_t* b_ring = smem + SA * L::kAPad;
+    __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(b_ring + UB * L::kUnitBytes);
+    int32_t* idx_buf = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(stage) + L::kStageBytes);
+    uint8_t* tile_ring = reinterpret_cast<uint8_t*>(idx_buf + kIdxBufs * p.idx_buf_elems);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(tile_ring + kTileSlots * kSlotBytes);
+    int* misc = reinterpret_cast<int*>(bars + L::num_bars(SA, UB));
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
+    volatile int* abort_flag = misc + 1;
+
+    const uint32_t fullA0 = smem_addr(bars), emptyA0 = fullA0 + 8 * SA;
+    const uint32_t fullB0 = emptyA0 + 8 * SA, emptyB0 = fullB0 + 8 * UB;
+    const uint32_t accF0 = emptyB0 + 8 * UB, accE0 = accF0 + 8 * kAccBufs;
+    const uint32_t idxF0 = accE0 + 8 * kAccBufs, idxE0 = idxF0 + 8 * kIdxBufs;
+    const uint32_t tileF0 = idxE0 + 8 * kIdxBufs, tileE0 = tileF0 + 8 * kTileSlots;
+    const uint32_t drain = tileE0 + 8 * kTileSlots;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nchunks = p.cin / KC;
+    const int64_t units = p.tiles * p.cblocks;
+
+    if (threadIdx.x == kWarpTma * 32) {
+        for (int s = 0; s < SA; ++s) {
+            mbar_init(fullA0 + 8 * s, 1);
+            mbar_init(emptyA0 + 8 * s, 1);
+        }
+        for (int u = 0; u < UB; ++u) {
+            mbar_init(fullB0 + 8 * u, 32 * kGatherWarps);  // every lane of every gather warp
+            mbar_init(emptyB0 + 8 * u, 1);
+        }
+        for (int b = 0; b < kAccBufs; ++b) {
+            mbar_init(accF0 + 8 * b, 1);
+            mbar_init(accE0 + 8 * b, kEpiWarps);
+        }
+        for (int b = 0; b < kIdxBufs; ++b) {
+            mbar_init(idxF0 + 8 * b, 1);
+            mbar_init(idxE0 + 8 * b, kGatherWarps);
+        }
+        for (int s = 0; s < kTileSlots; ++s) {
+            mbar_init(tileF0 + 8 * s, 1);
+            mbar_init(tileE0 + 8 * s, kTileConsumers);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == kWarpMma) {
+        tmem_alloc(smem_addr(tmem_slot), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    bool aborted = false;
+
+    if (warp == kWarpMma) {
+        // ------------------------------------------------ tcgen05.mma issuer (lane 0)
+        if (lane == 0) {
+            int as = SA - 1;
+            uint32_t aph = 1u;
+            int ucur = 0;
+            uint32_t bph = 0;  // bit u: phase of unit u's next use
+            for (int i = 0; !aborted; ++i) {
+                const int s = i % kTileSlots;
+                const uint8_t* slot = tile_ring + s * kSlotBytes;
+                if (!wait_bar<kSleepMma>(tileF0 + 8 * s, (uint32_t)(i / kTileSlots) & 1u, abort_flag, p.err)) {
+                    aborted = true;
+                    break;
+                }
+                if (slot_unit(slot) < 0) break;
+                const uint32_t* rec = slot_rec(slot);
+                const int buf = i & 1;
+                if (!wait_bar<kSleepMma>(accE0 + 8 * buf, ((uint32_t)(i >> 1) & 1u) ^ 1u, abort_flag, p.err)) {
+                    aborted = true;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t dbase = tmem + (uint32_t)buf * kAccCols;
+                const int nj = (int)rec[0];
+                int prev_k = -1;
+                uint32_t jw = rec[kWinRecHeader];
+                for (int j = 0; j < nj && !aborted; ++j) {
+                    const uint32_t jn = j + 1 < nj ? rec[kWinRecHeader + j + 1] : 0xFFFFFFFFu;
+                    const int k = win_job_k(jw), w0 = win_job_w0(jw), ncols = win_job_nw(jw) * kWinCols;
+                    const bool new_k = k != prev_k;
+                    prev_k = k;
+                    const bool last_of_k = jn == 0xFFFFFFFFu || win_job_k(jn) != k;
+                    const uint32_t idesc = idesc_bf16(BM, (uint32_t)ncols);
+                    const uint32_t d = dbase + (uint32_t)(w0 * kWinCols);
+                    for (int c = 0; c < nchunks; ++c) {
+                        if (nchunks > 1 || (c == 0 && new_k)) {
+                            if (++as == SA) {
+                                as = 0;
+                                aph ^= 1u;
+                            }
+                            if (!wait_bar<kSleepMma>(fullA0 + 8 * as, aph, abort_flag, p.err)) {
+                                aborted = true;
+                                break;
+                            }
+                        }
+                        int m = 0;
+                        const int u0 = alloc_units(ucur, UB, ncols, &m);
+                        for (int q = 0; q < m; ++q) {
+                            if (!wait_bar<kSleepMma>(fullB0 + 8 * (u0 + q), (bph >> (u0 + q)) & 1u, abort_flag,
+                                                     p.err)) {
+                                aborted = true;
+                                break;
+                            }
+                        }
+                        if (aborted) break;
+                        // the B units were written by cp.async (generic proxy); the MMA
+                        // reads them through the async proxy
+                        fence_proxy_async_smem();
+                        // descriptors of K step 0; later steps add their byte offset (>> 4)
+                        // to the start-address field, which cannot carry out of it because
+                        // shared addresses stay below 256 KB
+                        const uint64_t adesc0 = smem_desc(smem_addr(a_ring + as * L::kAPad), KC * 128, 1024, 2);
+                        const uint64_t bdesc0 = smem_desc(smem_addr(b_ring) + (uint32_t)(u0 * L::kUnitAtomBytes), 16,
+                                                          L::kBSbo, L::kBLayout);
+#pragma unroll
+                        for (int kk = 0; kk < KC / 16; ++kk) {
+                            const uint32_t boff = (uint32_t)((kk / L::kStepsPerAtom) * UB * L::kUnitAtomBytes +
+                                                             (kk % L::kStepsPerAtom) * 32);
+                            mma_bf16(d, adesc0 + (uint64_t)((kk * 2048) >> 4), bdesc0 + (uint64_t)(boff >> 4), idesc,
+                                     (j == 0 && c == 0 && kk == 0) ? 0u : 1u);
+                        }
+                        for (int q = 0; q < m; ++q) {
+                            mma_commit(emptyB0 + 8 * (u0 + q));
+                            bph ^= 1u << (u0 + q);
+                        }
+                        if (nchunks > 1 || last_of_k) mma_commit(emptyA0 + 8 * as);
+                    }
+                    jw = jn;
+                }
+                if (aborted) break;
+                mma_commit(accF0 + 8 * buf);
+                mbar_arrive(tileE0 + 8 * s);
+            }
+            if (aborted) {
+                mma_commit(drain);  // wait for the MMAs in flight before TMEM is freed
+                const uint64_t t0 = globaltimer_ns();
+                while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == kWarpTma) {
+        // ------------------------------------------------ scheduler + weight tiles (lane 0)
+        if (lane == 0) {
+            // Claim unit number idx into slot idx % kTileSlots once all consumers have
+            // released that slot's previous unit; no unit left: a -1 marker.
+            auto push = [&](int idx) -> bool {
+                const int s = idx % kTileSlots;
+                uint8_t* slot = tile_ring + s * kSlotBytes;
+                if (!wait_bar<kSleepProducer>(tileE0 + 8 * s, ((uint32_t)(idx / kTileSlots) & 1u) ^ 1u, abort_flag,
+                                              p.err))
+                    return false;
+                const unsigned int c = atomicAdd(p.work, 1u);  // claim number: tile order, then channel block
+                int* su = reinterpret_cast<int*>(slot);
+                if ((int64_t)c >= units) {
+                    su[0] = -1;
+                    mbar_arrive(tileF0 + 8 * s);
+                    return false;
+                }
+                const int64_t t = p.order ? (int64_t)p.order[c / p.cblocks] : (int64_t)(c / p.cblocks);
+                su[0] = (int)t;
+                su[1] = (int)(c % p.cblocks);
+                if (p.recs) {
+                    mbar_arrive_expect_tx(tileF0 + 8 * s, kRecBytes);
+                    bulk_load(smem_addr(slot + 16), p.recs + t * kWinJobStride, kRecBytes, tileF0 + 8 * s);
+                } else {  // kernel size 1: one centre job over the tile, no index stream
+                    uint32_t* r = reinterpret_cast<uint32_t*>(slot + 16);
+                    r[0] = 1u;
+                    r[1] = 0u;
+                    r[kWinRecHeader] = win_job(0, 0, p.rows / kWinCols);
+                    mbar_arrive(tileF0 + 8 * s);
+                }
+                return true;
+            };
+            // claims run two units ahead of the weight loads
+            bool more = push(0) && push(1);
+            int s_a = 0;  // weight slot and phase
+            uint32_t ph = 0;
+            for (int i = 0; !aborted; ++i) {
+                if (more) more = push(i + 2);
+                if (*abort_flag) {
+                    aborted = true;
+                    break;
+                }
+                const int s = i % kTileSlots;
+                const uint8_t* slot = tile_ring + s * kSlotBytes;
+                if (!wait_bar<kSleepProducer>(tileF0 + 8 * s, (uint32_t)(i / kTileSlots) & 1u, abort_flag, p.err)) {
+                    aborted = true;
+                    break;
+                }
+                if (slot_unit(slot) < 0) break;
+                const int cblk = slot_cblk(slot);
+                const uint32_t* rec = slot_rec(slot);
+                const int nj = (int)rec[0];
+                int prev_k = -1;
+                for (int j = 0; j < nj && !aborted; ++j) {
+                    const int k = win_job_k(rec[kWinRecHeader + j]);
+                    const bool new_k = k != prev_k;
+                    prev_k = k;
+                    if (nchunks == 1 && !new_k) continue;  // the loaded tile serves this job too
+                    for (int c = 0; c < nchunks; ++c) {
+                        if (!wait_bar<kSleepProducer>(emptyA0 + 8 * s_a, ph ^ 1u, abort_flag, p.err)) {
+                            aborted = true;
+                            break;
+                        }
+                        const uint32_t dst = smem_addr(a_ring + s_a * L::kAPad);
+                        mbar_arrive_expect_tx(fullA0 + 8 * s_a, L::kABytes);
+                        const int y = k * p.cin + c * KC;
+                        for (int box = 0; box < BM / 64; ++box)
+                            tma_load_2d(dst + box * KC * 128, &wmap, cblk * BM + box * 64, y, fullA0 + 8 * s_a);
+                        if (++s_a == SA) {
+                            s_a = 0;
+                            ph ^= 1u;
+                        }
+                    }
+                }
+            }
+            if (aborted) __nanosleep(200000);  // let loads in flight land before the CTA exits
+        }
+        __syncwarp();
+    } else if (warp < kWarpEpi0) {
+        // ------------------------------------------------ gather producers
+        // Gather warp g fills rows [16 g, 16 g + 16) of every unit.  Lane l copies
+        // 16-byte chunk l % kThreadsPerRow of rows l / kThreadsPerRow + kWarpRows *
+        // pass.  The source rows of all passes are read first (rows past the job
+        // read as holes, so no pass branches), then every pass issues its copy.
+        const int g = warp - kWarpGather0;
+        const int q = lane % L::kThreadsPerRow;
+        const int prow = lane / L::kThreadsPerRow;
+        const int atom = q / L::kChunksPerAtom, qa = q % L::kChunksPerAtom;
+        const bool issuer = g == 0 && p.idx_stream != nullptr;  // fetches the index streams
+        int ucur = 0;
+        uint32_t bph = 0;
+        // the index stream of tile number i goes to buffer i & 1, free once every
+        // gather warp has finished tile number i - 2
+        auto fetch_idx = [&](int i) -> bool {
+            const int s = i % kTileSlots;
+            const uint8_t* slot = tile_ring + s * kSlotBytes;
+            if (!warp_wait_bar<kSleepProducer>(tileF0 + 8 * s, (uint32_t)(i / kTileSlots) & 1u, abort_flag, p.err))
+                return false;
+            if (slot_unit(slot) < 0) return true;  // no such tile
+            const int b = i & 1;
+            if (!warp_wait_bar<kSleepProducer>(idxE0 + 8 * b, ((uint32_t)(i >> 1) & 1u) ^ 1u, abort_flag, p.err))
+                return false;
+            if (lane == 0) {
+                const uint32_t* rec = slot_rec(slot);
+                const uint32_t bytes = rec[1] * 4u;
+                const int64_t s0 = (int64_t)((uint64_t)rec[2] | ((uint64_t)rec[3] << 32));
+                mbar_arrive_expect_tx(idxF0 + 8 * b, bytes);
+                bulk_load(smem_addr(idx_buf + b * p.idx_buf_elems), p.idx_stream + s0, bytes, idxF0 + 8 * b);
+            }
+            __syncwarp();
+            return true;
+        };
+        if (issuer && !fetch_idx(0)) aborted = true;
+        for (int i = 0; !aborted; ++i) {
+            const int s = i % kTileSlots;
+            const uint8_t* slot = tile_ring + s * kSlotBytes;
+            if (!warp_wait_bar<kSleepProducer>(tileF0 + 8 * s, (uint32_t)(i / kTileSlots) & 1u, abort_flag, p.err)) {
+                aborted = true;
+                break;
+            }
+            const int u = slot_unit(slot);
+            if (u < 0) break;
+            if (issuer && !fetch_idx(i + 1)) {
+                aborted = true;
+                break;
+            }
+            const int buf = i & 1;
+            if (p.idx_stream &&
+                !warp_wait_bar<kSleepProducer>(idxF0 + 8 * buf, (uint32_t)(i >> 1) & 1u, abort_flag, p.err)) {
+                aborted = true;
+                break;
+            }
+            const int32_t* ibuf = idx_buf + buf * p.idx_buf_elems;
+            const int64_t row_t0 = (int64_t)u * p.rows;
+            const uint32_t* rec = slot_rec(slot);
+            const int nj = (int)rec[0];
+            int joff = 0;  // the job's first entry in the tile's index stream
+            for (int j = 0; j < nj && !aborted; ++j) {
+                const uint32_t jw = rec[kWinRecHeader + j];
+                const int ncols = win_job_nw(jw) * kWinCols;
+                const int64_t r0 = row_t0 + win_job_w0(jw) * kWinCols;  // first sorted row of the job
+                for (int c = 0; c < nchunks && !aborted; ++c) {
+                    int m = 0;
+                    const int u0 = alloc_units(ucur, UB, ncols, &m);
+                    const __nv_bfloat16* xc = p.x + c * KC + q * 8;
+                    for (int qq = 0; qq < m; ++qq) {
+                        const int unit = u0 + qq;
+                        if (!warp_wait_bar<kSleepProducer>(emptyB0 + 8 * unit, ((bph >> unit) & 1u) ^ 1u, abort_flag,
+                                                           p.err)) {
+                            aborted = true;
+                            break;
+                        }
+                        const int jr0 = qq * kUnitRows + g * L::kSliceRows;  // first job row of this slice
+                        int src[L::kPasses];
+#pragma unroll
+                        for (int pp = 0; pp < L::kPasses; ++pp) {
+                            const int r = jr0 + prow + pp * L::kWarpRows;  // job row
+                            if (p.idx_stream) {
+                                const int v = ibuf[joff + r];
+                                src[pp] = r < ncols ? v : -1;
+                            } else {
+                                const int64_t rr = r0 + r;
+                                src[pp] = r < ncols && rr < p.n ? (int)rr : -1;
+                            }
+                        }
+                        const uint32_t ubase = smem_addr(b_ring) + (uint32_t)(atom * UB * L::kUnitAtomBytes) +
+                                               (uint32_t)(unit * L::kUnitAtomBytes);
+#pragma unroll
+                        for (int pp = 0; pp < L::kPasses; ++pp) {
+                            const uint32_t lin =
+                                (uint32_t)((g * L::kSliceRows + prow + pp * L::kWarpRows) * L::kARB + qa * 16);
+                            cp_async_16(ubase + (lin ^ (((lin >> 7) & L::kSwz) << 4)),
+                                        xc + (int64_t)(src[pp] >= 0 ? src[pp] : 0) * p.cin, src[pp] >= 0 ? 16u : 0u);
+                        }
+                        cp_async_mbar_arrive_noinc(fullB0 + 8 * unit);
+                    }
+                    for (int qq = 0; qq < m; ++qq) bph ^= 1u << (u0 + qq);
+                }
+                joff += ncols;
+            }
+            __syncwarp();
+            if (lane == 0) {
+                if (p.idx_stream) mbar_arrive(idxE0 + 8 * buf);  // this warp is done with the tile's indices
+                mbar_arrive(tileE0 + 8 * s);
+            }
+        }
+        if (issuer && aborted && lane == 0) __nanosleep(200000);  // the index copy in flight lands first
+        cp_async_wait_all();
+    } else {
+        // ------------------------------------------------ epilogue
+        const int quarter = warp & 3;
+        const int half = (warp - kWarpEpi0) >> 2;
+        const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
+        __nv_bfloat16* stg = stage + (warp - kWarpEpi0) * L::kStageRows * L::kChPerWarp;
+        constexpr int kVecPerRow = L::kChPerWarp * 2 / 16;
+        constexpr int kChunksPerWarp = kWinMaxRows / 32 / 2;  // this warp's 32-column chunks of a tile
+        const bool lane_ok = lane < L::kChPerWarp;
+        for (int i = 0; !aborted; ++i) {
+            const int s = i % kTileSlots;
+            const uint8_t* slot = tile_ring + s * kSlotBytes;
+            if (!warp_wait_bar<kSleepEpilogue>(tileF0 + 8 * s, (uint32_t)(i / kTileSlots) & 1u, abort_flag, p.err)) {
+                aborted = true;
+                break;
+            }
+            const int u = slot_unit(slot);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tileE0 + 8 * s);  // only the unit number is needed here
+            if (u < 0) break;
+            const int64_t t = u;
+            const int cblk = slot_cblk(slot);
+            const int buf = i & 1;
+            const int ch_base = cblk * BM + quarter * L::kChPerWarp;
+            const int64_t row_t0 = t * p.rows;
+            const int t_eff = (int)min((int64_t)p.rows, p.n - row_t0);
+            // output rows and bias first: their loads overlap the wait for the MMAs
+            // (columns at or past t_eff are not this tile's rows)
+            int orow[kChunksPerWarp];
+#pragma unroll
+            for (int c4 = 0; c4 < kChunksPerWarp; ++c4) {
+                const int col = (half + 2 * c4) * 32 + lane;
+                orow[c4] = col < t_eff ? (p.perm ? p.perm[row_t0 + col] : (int)(row_t0 + col)) : -1;
+            }
+            const float bv = (p.bias && lane_ok) ? __bfloat162float(p.bias[ch_base + lane]) : 0.0f;
+            if (!warp_wait_bar<kSleepEpilogue>(accF0 + 8 * buf, (uint32_t)(i >> 1) & 1u, abort_flag, p.err)) {
+                aborted = true;
+                break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int c4 = 0; c4 < kChunksPerWarp; ++c4) {
+                const int cc = half + 2 * c4;
+                if (cc * 32 < t_eff) {
+                    float v[32];
+                    tmem_ld_x32(tmem + lane_base + (uint32_t)buf * kAccCols + (uint32_t)(cc * 32), v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int hp = 0; hp < 32 / L::kStageRows; ++hp) {
+                        if (lane_ok) {
+#pragma unroll
+                            for (int e = 0; e < L::kStageRows; ++e)
+                                stg[e * L::kChPerWarp + lane] = __float2bfloat16_rn(v[hp * L::kStageRows + e] + bv);
+                        }
+                        __syncwarp();
+#pragma unroll
+                        for (int e = lane; e < L::kStageRows * kVecPerRow; e += 32) {
+                            const int row = e / kVecPerRow, vq = e % kVecPerRow;
+                            const int o = __shfl_sync(0xffffffffu, orow[c4], hp * L::kStageRows + row);
+                            if (o >= 0) {
+                                const int4 val = *reinterpret_cast<const int4*>(stg + row * L::kChPerWarp + vq * 8);
+                                *reinterpret_cast<int4*>(p.out + (int64_t)o * p.cout + ch_base + vq * 8) = val;
+                            }
+                        }
+                        __syncwarp();
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(accE0 + 8 * buf);
+        }
+    }
+
+    // ---- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kWarpMma) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    });
+    return fn;
+}
+
+int g_force_sa = 0, g_force_ub = 0;  // test hook: ring depths (0 = automatic)
+
+// Ring depths: three weight slots (two if that leaves too few units), then as
+// many B units as fit (at most kMaxUnits), then any room left to weight slots (at
+// most kMaxASlots); a tile's centre job needs ceil(rows / 64) units at once.
+// max_cols sizes the two tile index buffers.
+template <int BM, int KC>
+bool choose_depths(int rows, int max_cols, int* sa, int* ub) {
+    using L = WinLayout<BM, KC>;
+    const int need = (rows + kUnitRows - 1) / kUnitRows;
+    if (g_force_sa > 0 && g_force_ub > 0) {
+        *sa = g_force_sa;
+        *ub = g_force_ub;
+        return *ub >= need && *ub <= kMaxUnits && *sa <= kMaxASlots && L::smem_bytes(*sa, *ub, max_cols) <= kMaxSmem;
+    }
+    for (int a = 3; a >= 2; --a) {
+        int b = 0;
+        while (b < kMaxUnits && L::smem_bytes(a, b + 1, max_cols) <= kMaxSmem) ++b;
+        if (b >= need + 1 || (a == 2 && b >= need)) {
+            while (a < kMaxASlots && L::smem_bytes(a + 1, b, max_cols) <= kMaxSmem) ++a;
+            *sa = a;
+            *ub = b;
+            return true;
+        }
+    }
+    return false;
+}
+
+template <int BM, int KC>
+spconv_status_t launch(const MapData& m, const void* x, int cin, const void* w, const void* bias, void* out,
+                       int cout, cudaStream_t stream, cudaError_t* ce) {
+    using L = WinLayout<BM, KC>;
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) {
+        *ce = cudaErrorSymbolNotFound;
+        return SPCONV_ERR_CUDA;
+    }
+    const int kvol = m.kernel_size == 3 ? kVol3 : 1;
+    const int max_cols = kvol == kVol3 ? (int)m.max_tile_cols : 0;
+    int sa = 0, ub = 0;
+    if (!choose_depths<BM, KC>(m.win_rows, max_cols, &sa, &ub)) return SPCONV_ERR_UNSUPPORTED;
+    // Weights [kvol, cin, cout] viewed as 2-D [kvol*cin rows, cout columns]; a box
+    // is 64 output channels (128 B, 128-byte swizzle) by KC input channels.
+    CUtensorMap map;
+    const cuuint64_t dims[2] = {(cuuint64_t)cout, (cuuint64_t)kvol * cin};
+    const cuuint64_t strides[1] = {(cuuint64_t)cout * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)KC};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(w), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        *ce = cudaErrorInvalidValue;
+        return SPCONV_ERR_CUDA;
+    }
+    const int need_smem = L::smem_bytes(sa, ub, max_cols);
+    const int smem = need_smem > kMinSmem ? need_smem : kMinSmem;
+    int dev = 0;
+    cudaError_t de = cudaGetDevice(&dev);
+    if (de != cudaSuccess) {
+        *ce = de;
+        return SPCONV_ERR_CUDA;
+    }
+    {   // the shared-memory opt-in is per device context and instantiation
+        static std::mutex attr_mu;
+        static std::vector<char> attr_done;
+        std::lock_guard<std::mutex> lock(attr_mu);
+        if (dev >= (int)attr_done.size()) attr_done.resize((size_t)dev + 1, 0);
+        if (!attr_done[dev]) {
+            const cudaError_t ae =
+                cudaFuncSetAttribute(k_subm_win<BM, KC>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+            if (ae != cudaSuccess) {
+                *ce = ae;
+                return SPCONV_ERR_CUDA;
+            }
+            attr_done[dev] = 1;
+        }
+    }
+    // this launch's work counter: one of the map's slots, cleared on the stream
+    static std::atomic<uint64_t> launches{0};
+    unsigned int* work = m.sched + (launches.fetch_add(1) % kSchedSlots);
+    cudaError_t me = cudaMemsetAsync(work, 0, sizeof(unsigned int), stream);
+    if (me != cudaSuccess) {
+        *ce = me;
+        return SPCONV_ERR_CUDA;
+    }
+    WinParams p;
+    p.perm = kvol == kVol3 ? m.perm : nullptr;
+    p.recs = kvol == kVol3 ? m.win_jobs : nullptr;
+    p.idx_stream = kvol == kVol3 ? m.idx_stream : nullptr;
+    p.order = kvol == kVol3 ? m.win_order : nullptr;
+    p.work = work;
+    p.n = m.n;
+    p.tiles = m.win_tiles;
+    p.rows = m.win_rows;
+    p.cblocks = cout / BM;
+    p.x = static_cast<const __nv_bfloat16*>(x);
+    p.cin = cin;
+    p.bias = static_cast<const __nv_bfloat16*>(bias);
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.cout = cout;
+    p.err = m.fwd_err;
+    p.sa = sa;
+    p.ub = ub;
+    p.idx_buf_elems = L::idx_buf_bytes(max_cols) / 4;
+    const int64_t units = m.win_tiles * p.cblocks;
+    const int64_t grid = units < m.num_sms ? units : m.num_sms;
+    k_subm_win<BM, KC><<<(unsigned)grid, kThreads, smem, stream>>>(map, p);
+    *ce = cudaGetLastError();
+    return *ce == cudaSuccess ? SPCONV_OK : SPCONV_ERR_CUDA;
+}
+
+}  // namespace
+
+void set_forced_ring_depths(int sa, int ub) {
+    g_force_sa = sa;
+    g_force_ub = ub;
+}
+
+spconv_status_t launch_forward_tcgen05(const MapData& m, const void* x, int cin, const void* w, const void* bias,
+                                       void* out, int cout, cudaStream_t stream, cudaError_t* ce) {
+    *ce = cudaSuccess;
+    if (cin % 16 != 0 || cout % 64 != 0) return SPCONV_ERR_UNSUPPORTED;
+    if (m.n == 0) return SPCONV_OK;
+    const bool bm128 = cout % 128 == 0;
+    const int kc = cin % 128 == 0 ? 128 : (cin % 64 == 0 ? 64 : (cin % 32 == 0 ? 32 : 16));
+    if (bm128) {
+        if (kc == 128) return launch<128, 128>(m, x, cin, w, bias, out, cout, stream, ce);
+        if (kc == 64) return launch<128, 64>(m, x, cin, w, bias, out, cout, stream, ce);
+        if (kc == 32) return launch<128, 32>(m, x, cin, w, bias, out, cout, stream, ce);
+        return launch<128, 16>(m, x, cin, w, bias, out, cout, stream, ce);
+    }
+    if (kc == 128) return launch<64, 128>(m, x, cin, w, bias, out, cout, stream, ce);
+    if (kc == 64) return launch<64, 64>(m, x, cin, w, bias, out, cout, stream, ce);
+    if (kc == 32) return launch<64, 32>(m, x, cin, w, bias, out, cout, stream, ce);
+    return launch<64, 16>(m, x, cin, w, bias, out, cout, stream, ce);
+}
+
+}  // namespace spconv

@@ -59,47 +59,73 @@ __global__ void k_insert(const int4* __restrict__ coords, int64_t n, int ex, int
     atomicOr(&flags->err, kErrTableFull);
 }
 
-// One thread per (voxel i, offset k), k fastest, so the [n, 27] stores coalesce.
-__global__ void k_probe(const int4* __restrict__ coords, int64_t n, int ex, int ey, int ez,
-                        const ulonglong2* __restrict__ table, unsigned long long mask,
-                        int32_t* __restrict__ nbr, BuildFlags* __restrict__ flags) {
-    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    bool hit = false;
-    if (t < n * kVol3) {
-        const int64_t i = t / kVol3;
-        const int k = (int)(t - i * kVol3);
-        int32_t found = -1;
-        if (k == kCentre) {
-            found = (int32_t)i;
-        } else {
-            const int4 c = coords[i];
-            const int x = c.y + k / 9 - 1, y = c.z + (k / 3) % 3 - 1, z = c.w + k % 3 - 1;
-            if ((unsigned)x < (unsigned)ex && (unsigned)y < (unsigned)ey && (unsigned)z < (unsigned)ez) {
-                const unsigned long long key = pack_key(c.x, x, y, z);
-                unsigned long long slot = mix64(key) & mask;
-                for (unsigned long long it = 0; it <= mask; ++it) {
-                    const ulonglong2 s = table[slot];
-                    if (s.x == key) {
-                        found = (int32_t)s.y;
-                        break;
+// Rank of a mask in the reflected Gray-code sequence (the inverse Gray code):
+// sorting by it puts masks that differ in few bits next to each other.
+__device__ __forceinline__ uint32_t gray_rank(uint32_t g) {
+    g ^= g >> 1;
+    g ^= g >> 2;
+    g ^= g >> 4;
+    g ^= g >> 8;
+    g ^= g >> 16;
+    return g;
+}
+
+constexpr int kProbeThreads = 128;
+
+// One thread per voxel: its coordinate is read once and its 26 neighbours are
+// probed in turn.  The [rows, 27] results are staged in shared memory so the
+// block's stores to the map are contiguous.  Optionally writes the sort key of
+// the row: the Gray rank of its 26 non-centre hit bits (offset k, centre
+// skipped, is bit 25 - ks with ks = k < 13 ? k : k - 1).
+__global__ void __launch_bounds__(kProbeThreads)
+    k_probe_rows(const int4* __restrict__ coords, int64_t n, int ex, int ey, int ez,
+                 const ulonglong2* __restrict__ table, unsigned long long mask, int32_t* __restrict__ nbr,
+                 uint32_t* __restrict__ keys, BuildFlags* __restrict__ flags) {
+    __shared__ int32_t stage[kProbeThreads * kVol3];
+    const int64_t i0 = (int64_t)blockIdx.x * kProbeThreads;
+    const int64_t i = i0 + threadIdx.x;
+    uint32_t bits = 0;
+    int hits = 0;
+    if (i < n) {
+        const int4 c = coords[i];
+        for (int k = 0; k < kVol3; ++k) {
+            int32_t found = -1;
+            if (k == kCentre) {
+                found = (int32_t)i;
+            } else {
+                const int x = c.y + k / 9 - 1, y = c.z + (k / 3) % 3 - 1, z = c.w + k % 3 - 1;
+                if ((unsigned)x < (unsigned)ex && (unsigned)y < (unsigned)ey && (unsigned)z < (unsigned)ez) {
+                    const unsigned long long key = pack_key(c.x, x, y, z);
+                    unsigned long long slot = mix64(key) & mask;
+                    for (unsigned long long it = 0; it <= mask; ++it) {
+                        const ulonglong2 s = table[slot];
+                        if (s.x == key) {
+                            found = (int32_t)s.y;
+                            break;
+                        }
+                        if (s.x == kEmptyKey) break;
+                        slot = (slot + 1) & mask;
                     }
-                    if (s.x == kEmptyKey) break;
-                    slot = (slot + 1) & mask;
                 }
+                if (found >= 0) bits |= 1u << (25 - (k < kCentre ? k : k - 1));
             }
+            hits += found >= 0 ? 1 : 0;
+            stage[threadIdx.x * kVol3 + k] = found;
         }
-        nbr[t] = found;
-        hit = found >= 0;
+        if (keys) keys[i] = gray_rank(bits);
     }
-    const unsigned ballot = __ballot_sync(0xffffffffu, hit);
-    if ((threadIdx.x & 31) == 0 && ballot) atomicAdd(&flags->pairs, (unsigned long long)__popc(ballot));
+    __syncthreads();
+    const int rows = (int)min((int64_t)kProbeThreads, n - i0);
+    for (int e = threadIdx.x; e < rows * kVol3; e += kProbeThreads) nbr[i0 * kVol3 + e] = stage[e];
+    for (int d = 16; d > 0; d >>= 1) hits += __shfl_down_sync(0xffffffffu, hits, d);
+    if ((threadIdx.x & 31) == 0 && hits) atomicAdd(&flags->pairs, (unsigned long long)hits);
 }
 
 }  // namespace
 
 cudaError_t launch_build_map(const int32_t* coords, int64_t n, const int32_t extent[3], int32_t kernel_size,
-                             unsigned long long* table, uint64_t slots, int32_t* nbr, BuildFlags* flags,
-                             cudaStream_t stream) {
+                             unsigned long long* table, uint64_t slots, int32_t* nbr, uint32_t* keys,
+                             BuildFlags* flags, cudaStream_t stream) {
     cudaError_t e = cudaMemsetAsync(table, 0xFF, slots * 16, stream);
     if (e != cudaSuccess) return e;
     e = cudaMemsetAsync(flags, 0, sizeof(BuildFlags), stream);
@@ -111,167 +137,9 @@ cudaError_t launch_build_map(const int32_t* coords, int64_t n, const int32_t ext
         c4, n, extent[0], extent[1], extent[2], table, slots - 1, flags);
     e = cudaGetLastError();
     if (e != cudaSuccess || kernel_size == 1) return e;
-    const int64_t work = n * kVol3;
-    k_probe<<<(unsigned)((work + threads - 1) / threads), threads, 0, stream>>>(
-        c4, n, extent[0], extent[1], extent[2], reinterpret_cast<const ulonglong2*>(table), slots - 1, nbr,
+    k_probe_rows<<<(unsigned)((n + kProbeThreads - 1) / kProbeThreads), kProbeThreads, 0, stream>>>(
+        c4, n, extent[0], extent[1], extent[2], reinterpret_cast<const ulonglong2*>(table), slots - 1, nbr, keys,
         flags);
-    return cudaGetLastError();
-}
-
-}  // namespace spconv
-
-// ---------------------------------------------------------------------------
-// Tile metadata.  One CTA per tile stages the tile's [rows, 27] map rows in
-// shared memory (coalesced), then warps scan the (offset, class) units with
-// ballots: k_tile_count writes the per-unit counts and the tile's padded entry
-// total; k_tile_scan turns the totals into offsets; k_tile_fill writes the
-// entries (local row, neighbour row) in unit order, rows ascending per unit.
-namespace spconv {
-namespace {
-
-constexpr int kMetaThreads = 256;
-
-__device__ __forceinline__ void stage_tile_rows(const int32_t* __restrict__ nbr, int64_t row0, int t_eff,
-                                                int32_t* __restrict__ tile_s) {
-    const int words = t_eff * kVol3;
-    const int32_t* src = nbr + row0 * kVol3;
-    for (int i = threadIdx.x; i < words; i += blockDim.x) tile_s[i] = __ldg(src + i);
-}
-
-__device__ __forceinline__ int unit_offset(int u) {
-    const int ks = u / kTileClasses;
-    return ks < kCentre ? ks : ks + 1;
-}
-
-__global__ void k_tile_count(const int32_t* __restrict__ nbr, int64_t n, int tile_rows,
-                             int32_t* __restrict__ tile_counts, int64_t* __restrict__ tile_total) {
-    __shared__ int32_t tile_s[kTileRows * kVol3];
-    __shared__ int32_t cnt_s[kTileUnits];
-    const int64_t t = blockIdx.x;
-    const int64_t row0 = t * tile_rows;
-    const int t_eff = (int)min((int64_t)tile_rows, n - row0);
-    stage_tile_rows(nbr, row0, t_eff, tile_s);
-    __syncthreads();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int u = warp; u < kTileUnits; u += kMetaThreads / 32) {
-        const int k = unit_offset(u), c = u % kTileClasses;
-        int count = 0;
-        for (int base = 0; base < kTileRows / kTileClasses; base += 32) {
-            const int r = c + kTileClasses * (base + lane);
-            const bool hit = r < t_eff && tile_s[r * kVol3 + k] >= 0;
-            count += __popc(__ballot_sync(0xffffffffu, hit));
-        }
-        if (lane == 0) cnt_s[u] = count;
-    }
-    __syncthreads();
-    if (threadIdx.x < kTileCountStride)
-        tile_counts[t * kTileCountStride + threadIdx.x] = threadIdx.x < kTileUnits ? cnt_s[threadIdx.x] : 0;
-    if (threadIdx.x == 0) {
-        int64_t total = 0;
-        for (int u = 0; u < kTileUnits; ++u) total += cnt_s[u];
-        tile_total[t] = (total + kTileEntryAlign - 1) / kTileEntryAlign * kTileEntryAlign;
-    }
-}
-
-// Exclusive scan of the per-tile totals (in place, one CTA): off[t] = sum of
-// totals before t; off[ntiles] = grand total; off[ntiles + 1] = largest total
-// of one tile (the forward kernel sizes its shared-memory entry lists by it).
-__global__ void k_tile_scan(int64_t* __restrict__ off, int64_t ntiles) {
-    __shared__ int64_t part[1024];
-    __shared__ int64_t pmax[1024];
-    const int64_t per = (ntiles + blockDim.x - 1) / blockDim.x;
-    const int64_t lo = threadIdx.x * per, hi = min(ntiles, lo + per);
-    int64_t sum = 0, mx = 0;
-    for (int64_t i = lo; i < hi; ++i) {
-        sum += off[i];
-        mx = max(mx, off[i]);
-    }
-    part[threadIdx.x] = sum;
-    pmax[threadIdx.x] = mx;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int64_t run = 0, m = 0;
-        for (int i = 0; i < (int)blockDim.x; ++i) {
-            const int64_t v = part[i];
-            part[i] = run;
-            run += v;
-            m = max(m, pmax[i]);
-        }
-        off[ntiles] = run;
-        off[ntiles + 1] = m;
-    }
-    __syncthreads();
-    int64_t run = part[threadIdx.x];
-    for (int64_t i = lo; i < hi; ++i) {
-        const int64_t v = off[i];
-        off[i] = run;
-        run += v;
-    }
-}
-
-__global__ void k_tile_fill(const int32_t* __restrict__ nbr, int64_t n, int tile_rows,
-                            const int32_t* __restrict__ tile_counts,
-                            const int64_t* __restrict__ tile_off, uint16_t* __restrict__ pair_r,
-                            int32_t* __restrict__ pair_j) {
-    __shared__ int32_t tile_s[kTileRows * kVol3];
-    __shared__ int32_t start_s[kTileUnits];
-    const int64_t t = blockIdx.x;
-    const int64_t row0 = t * tile_rows;
-    const int t_eff = (int)min((int64_t)tile_rows, n - row0);
-    stage_tile_rows(nbr, row0, t_eff, tile_s);
-    if (threadIdx.x == 0) {
-        int run = 0;
-        for (int u = 0; u < kTileUnits; ++u) {
-            start_s[u] = run;
-            run += tile_counts[t * kTileCountStride + u];
-        }
-        // zero the padding entries of this tile
-        const int64_t end = tile_off[t + 1];
-        for (int64_t e = tile_off[t] + run; e < end; ++e) {
-            pair_r[e] = 0;
-            pair_j[e] = 0;
-        }
-    }
-    __syncthreads();
-    const int64_t base = tile_off[t];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int u = warp; u < kTileUnits; u += kMetaThreads / 32) {
-        const int k = unit_offset(u), c = u % kTileClasses;
-        int pos = start_s[u];
-        for (int b = 0; b < kTileRows / kTileClasses; b += 32) {
-            const int r = c + kTileClasses * (b + lane);
-            const int32_t j = r < t_eff ? tile_s[r * kVol3 + k] : -1;
-            const unsigned m = __ballot_sync(0xffffffffu, j >= 0);
-            if (j >= 0) {
-                const int64_t e = base + pos + __popc(m & ((1u << lane) - 1u));
-                pair_r[e] = (uint16_t)r;
-                pair_j[e] = j;
-            }
-            pos += __popc(m);
-        }
-    }
-}
-
-}  // namespace
-
-cudaError_t launch_tile_count(const int32_t* nbr, int64_t n, int tile_rows, int32_t* tile_counts, int64_t* tile_off,
-                              cudaStream_t stream) {
-    if (tile_rows < 1 || tile_rows > kTileRows) return cudaErrorInvalidValue;
-    const int64_t nt = num_tiles(n, tile_rows);
-    if (nt == 0) return cudaMemsetAsync(tile_off, 0, 2 * sizeof(int64_t), stream);
-    k_tile_count<<<(unsigned)nt, kMetaThreads, 0, stream>>>(nbr, n, tile_rows, tile_counts, tile_off);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    k_tile_scan<<<1, 1024, 0, stream>>>(tile_off, nt);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_tile_fill(const int32_t* nbr, int64_t n, int tile_rows, const int32_t* tile_counts,
-                             const int64_t* tile_off, uint16_t* pair_r, int32_t* pair_j, cudaStream_t stream) {
-    if (tile_rows < 1 || tile_rows > kTileRows) return cudaErrorInvalidValue;
-    const int64_t nt = num_tiles(n, tile_rows);
-    if (nt == 0) return cudaSuccess;
-    k_tile_fill<<<(unsigned)nt, kMetaThreads, 0, stream>>>(nbr, n, tile_rows, tile_counts, tile_off, pair_r, pair_j);
     return cudaGetLastError();
 }
 

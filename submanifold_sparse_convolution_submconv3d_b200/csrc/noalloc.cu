@@ -8,7 +8,6 @@
 // spconv_build_neighbor_map_noalloc serves them: the caller passes the output
 // buffer, and the hash table and error flags live in the file-scope array below,
 // which every GPU that loads this library holds until the process exits.
-#include <mutex>
 #include <string>
 
 #include "common.cuh"
@@ -24,31 +23,20 @@ constexpr size_t kNoAllocBytes = kNoAllocTableBytes + 256;  // + BuildFlags, 256
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mutex;
-unsigned char* g_scratch_ptr[kMaxDevices] = {};
-
 spconv_status_t noalloc_fail(spconv_status_t s, const std::string& msg) {
     spconv::set_last_error(msg);
     return s;
 }
 
-// Device address of the scratch array on the current device, looked up once per
-// device (the first call on a device does this; it should come before any
-// stream capture).
+// Device address of the scratch array on the current device.  In host code the
+// array's name only stands in for it, so the address is asked of the runtime with
+// the device current.  It is looked up on every call (the lookup allocates
+// nothing): a cached address would go stale if the device's context were reset.
 cudaError_t scratch_for_current_device(unsigned char** out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_mutex);
-    if (!g_scratch_ptr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_ptr[dev] = static_cast<unsigned char*>(p);
-    }
-    *out = g_scratch_ptr[dev];
+    *out = static_cast<unsigned char*>(p);
     return cudaSuccess;
 }
 
@@ -83,7 +71,7 @@ spconv_status_t spconv_build_neighbor_map_noalloc(const int32_t* coords, int64_t
     // previous call's contents).  Slots: power of two >= 2n, at most the array.
     uint64_t slots = 64;
     while (slots < (uint64_t)n * 2) slots <<= 1;
-    e = spconv::launch_build_map(coords, n, extent, 3, table, slots, nbr_out, flags, stream);
+    e = spconv::launch_build_map(coords, n, extent, 3, table, slots, nbr_out, nullptr, flags, stream);
     spconv::BuildFlags host_flags{};
     if (e == cudaSuccess) e = cudaMemcpyAsync(&host_flags, flags, sizeof(host_flags), cudaMemcpyDeviceToHost, stream);
     if (e == cudaSuccess) e = cudaStreamSynchronize(stream);

@@ -1,6 +1,6 @@
 // Thin inline-PTX wrappers for the sm_100a features the tensor-core forward uses:
-// mbarriers, cp.async gathers, TMA tiled loads, tensor memory (TMEM) allocation,
-// loads and stores, and tcgen05.mma / tcgen05.commit.  No multicast form of any
+// mbarriers, cp.async gathers, TMA tiled and bulk loads, tensor memory (TMEM)
+// allocation, loads and stores, and tcgen05.mma / tcgen05.commit.  No multicast form of any
 // load is used anywhere in this library.
 #pragma once
 
@@ -83,6 +83,14 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
             dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
         : "memory");
+}
+
+// One-dimensional bulk copy global -> this CTA's shared memory, completion counted
+// in bytes on `bar` (no multicast).  Addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
 }
 
 // ---------------------------------------------------------------- TMEM

@@ -1,11 +1,22 @@
 // C ABI of the SubMConv3d library: validation, the map handle, dispatch.
-#include <string>
+//
+// Device memory of the maps comes from one stream-ordered memory pool per device
+// that the library owns (cudaMallocFromPoolAsync on the build's stream).  The pool
+// keeps freed memory for reuse, so a map build after the first one maps no new
+// memory and never synchronises the device; the build synchronises its stream
+// once, at the end, to read back the device error flags.
+#include <atomic>
+#include <mutex>
 #include <new>
+#include <string>
+#include <vector>
 
 #include "common.cuh"
 
 struct spconv_map_s {
     spconv::MapData d;
+    std::atomic<int64_t> launches[SPCONV_KERNEL_KINDS] = {};  // forward launches per kernel family
+    std::vector<void*> owned;                                  // pool allocations the map owns
 };
 
 namespace {
@@ -32,6 +43,59 @@ uint64_t next_pow2(uint64_t v) {
     return p;
 }
 
+// The library's memory pool of device `dev`, created on first use.  Its release
+// threshold is the maximum, so memory freed to it stays mapped for later builds.
+cudaError_t device_pool(int dev, cudaMemPool_t* out) {
+    static std::mutex mu;
+    static std::vector<cudaMemPool_t> pools;
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 0) return cudaErrorInvalidDevice;
+    if (dev >= (int)pools.size()) pools.resize((size_t)dev + 1, nullptr);
+    if (!pools[dev]) {
+        cudaMemPoolProps props = {};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t pool = nullptr;
+        cudaError_t e = cudaMemPoolCreate(&pool, &props);
+        if (e != cudaSuccess) return e;
+        uint64_t threshold = ~0ull;
+        e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &threshold);
+        if (e != cudaSuccess) {
+            cudaMemPoolDestroy(pool);
+            return e;
+        }
+        pools[dev] = pool;
+    }
+    *out = pools[dev];
+    return cudaSuccess;
+}
+
+// Stream-ordered allocations of one build: the map's own buffers and transient
+// scratch, released on the build's stream.
+struct BuildAlloc {
+    cudaMemPool_t pool = nullptr;
+    cudaStream_t stream = nullptr;
+    std::vector<void*> scratch;
+    cudaError_t err = cudaSuccess;
+
+    template <typename T>
+    T* get(size_t count, std::vector<void*>& owner) {
+        if (err != cudaSuccess) return nullptr;
+        void* p = nullptr;
+        err = cudaMallocFromPoolAsync(&p, count > 0 ? count * sizeof(T) : 16, pool, stream);
+        if (err != cudaSuccess) return nullptr;
+        owner.push_back(p);
+        return static_cast<T*>(p);
+    }
+    template <typename T>
+    T* temp(size_t count) { return get<T>(count, scratch); }
+    void release_scratch() {
+        for (void* p : scratch) cudaFreeAsync(p, stream);
+        scratch.clear();
+    }
+};
+
 }  // namespace
 
 namespace spconv {
@@ -50,15 +114,42 @@ spconv_status_t spconv_debug_set_table_slots(int64_t slots) {
 
 spconv_status_t spconv_map_tile_rows(spconv_map_t map, int32_t* rows) {
     if (!map || !rows) return fail(SPCONV_ERR_INVALID_ARG, "null map or rows");
-    *rows = map->d.tile_rows;
+    *rows = map->d.win_rows;
     return SPCONV_OK;
 }
 
 spconv_status_t spconv_debug_set_tile_rows(int32_t rows) {
-    if (rows < 0 || rows > spconv::kTileRows) return fail(SPCONV_ERR_INVALID_ARG, "rows must be in [0, 384]");
+    if (rows < 0 || rows > spconv::kWinMaxRows || rows % spconv::kWinCols != 0)
+        return fail(SPCONV_ERR_INVALID_ARG, "rows must be 0 or a multiple of 16 in [16, 256]");
     g_tile_rows_override = rows;
     return SPCONV_OK;
 }
+
+spconv_status_t spconv_debug_set_ring_depths(int32_t a_slots, int32_t b_units) {
+    const bool auto_ = a_slots == 0 && b_units == 0;
+    if (!auto_ && (a_slots < 2 || a_slots > 8 || b_units < 4 || b_units > 32))
+        return fail(SPCONV_ERR_INVALID_ARG, "a_slots must be in [2, 8] and b_units in [4, 32], or both 0");
+    spconv::set_forced_ring_depths(a_slots, b_units);
+    return SPCONV_OK;
+}
+
+spconv_status_t spconv_free(spconv_map_t map) {
+    if (!map) return SPCONV_OK;
+    int prev = -1;
+    const bool have_prev = cudaGetDevice(&prev) == cudaSuccess;
+    if (map->d.device != prev) cudaSetDevice(map->d.device);
+    // Kernels on any stream may still read the map: wait for the device, then
+    // hand the memory back to the pool.
+    cudaDeviceSynchronize();
+    for (void* p : map->owned) cudaFreeAsync(p, nullptr);
+    if (have_prev && map->d.device != prev) cudaSetDevice(prev);
+    delete map;
+    return SPCONV_OK;
+}
+
+}  // extern "C"
+
+extern "C" {
 
 spconv_status_t spconv_build_map(const int32_t* coords, int64_t n, const int32_t* extent, int32_t kernel_size,
                                  void* stream_, spconv_map_t* out_map) {
@@ -73,56 +164,76 @@ spconv_status_t spconv_build_map(const int32_t* coords, int64_t n, const int32_t
 
     spconv_map_s* m = new (std::nothrow) spconv_map_s();
     if (!m) return fail(SPCONV_ERR_OOM, "host allocation failed");
-    m->d.n = n;
-    m->d.kernel_size = kernel_size;
-    for (int a = 0; a < 3; ++a) m->d.extent[a] = extent[a];
-    cudaError_t e = cudaGetDevice(&m->d.device);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&m->d.num_sms, cudaDevAttrMultiProcessorCount, m->d.device);
-    if (e == cudaSuccess) e = cudaMalloc(&m->d.fwd_err, sizeof(unsigned int));
-    if (e == cudaSuccess) e = cudaMemsetAsync(m->d.fwd_err, 0, sizeof(unsigned int), stream);
+    spconv::MapData& d = m->d;
+    d.n = n;
+    d.kernel_size = kernel_size;
+    for (int a = 0; a < 3; ++a) d.extent[a] = extent[a];
+    BuildAlloc al;
+    al.stream = stream;
+    cudaError_t e = cudaGetDevice(&d.device);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, d.device);
+    if (e == cudaSuccess) e = device_pool(d.device, &al.pool);
     if (e != cudaSuccess) {
-        cudaFree(m->d.fwd_err);
         delete m;
         return fail_cuda(e, "spconv_build_map setup");
     }
 
-    uint64_t slots = g_table_slots_override > 0 ? (uint64_t)g_table_slots_override
-                                                : next_pow2(n * 2 > 64 ? (uint64_t)n * 2 : 64);
-    unsigned long long* table = nullptr;
-    spconv::BuildFlags* flags = nullptr;
+    // Every size below follows from n, so all buffers are requested up front and
+    // the build needs a single synchronisation at its end.
+    d.win_rows = g_tile_rows_override > 0 ? g_tile_rows_override : spconv::choose_win_rows(n, d.num_sms);
+    d.win_tiles = (n + d.win_rows - 1) / d.win_rows;
+    d.npad = d.win_tiles * d.win_rows;
+    const bool k3 = kernel_size == 3 && n > 0;
+    const uint64_t slots = g_table_slots_override > 0 ? (uint64_t)g_table_slots_override
+                                                      : next_pow2(n * 2 > 64 ? (uint64_t)n * 2 : 64);
+    d.fwd_err = al.get<unsigned int>(1, m->owned);
+    d.sched = al.get<uint32_t>(spconv::kSchedSlots, m->owned);
+    auto* flags = al.temp<spconv::BuildFlags>(1);
     spconv::BuildFlags host_flags{};
-    spconv_status_t status = SPCONV_OK;
-    e = cudaMalloc(&table, slots * 16);
-    if (e == cudaSuccess) e = cudaMalloc(&flags, sizeof(spconv::BuildFlags));
-    if (e == cudaSuccess && kernel_size == 3 && n > 0) e = cudaMalloc(&m->d.nbr, (size_t)n * spconv::kVol3 * sizeof(int32_t));
-    m->d.tile_rows = g_tile_rows_override > 0 ? g_tile_rows_override : spconv::choose_tile_rows(n, m->d.num_sms);
-    const int64_t ntiles = spconv::num_tiles(n, m->d.tile_rows);
-    const bool tiles = kernel_size == 3 && n > 0;
-    if (e == cudaSuccess && tiles) e = cudaMalloc(&m->d.tile_counts, (size_t)ntiles * spconv::kTileCountStride * 4);
-    if (e == cudaSuccess && tiles) e = cudaMalloc(&m->d.tile_off, (size_t)(ntiles + 2) * sizeof(int64_t));
-    if (e == cudaSuccess)
-        e = spconv::launch_build_map(coords, n, extent, kernel_size, table, slots, m->d.nbr, flags, stream);
-    if (e == cudaSuccess && tiles)
-        e = spconv::launch_tile_count(m->d.nbr, n, m->d.tile_rows, m->d.tile_counts, m->d.tile_off, stream);
-    int64_t entry_stats[2] = {0, 0};  // grand total, largest tile
-    if (e == cudaSuccess && tiles)
-        e = cudaMemcpyAsync(entry_stats, m->d.tile_off + ntiles, sizeof(entry_stats), cudaMemcpyDeviceToHost, stream);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(&host_flags, flags, sizeof(host_flags), cudaMemcpyDeviceToHost, stream);
-    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
-    // Second phase (only if the map is valid): entry arrays of the tile metadata.
-    // entry_stats and host_flags are read only after the synchronisation above.
-    if (e == cudaSuccess && tiles && host_flags.err == 0) {
-        const int64_t total_entries = entry_stats[0];
-        m->d.tile_entries = total_entries;
-        m->d.tile_max_entries = entry_stats[1];
-        const size_t ne = total_entries > 0 ? (size_t)total_entries : 1;
-        e = cudaMalloc(&m->d.pair_r, ne * sizeof(uint16_t));
-        if (e == cudaSuccess) e = cudaMalloc(&m->d.pair_j, ne * sizeof(int32_t));
-        if (e == cudaSuccess)
-            e = spconv::launch_tile_fill(m->d.nbr, n, m->d.tile_rows, m->d.tile_counts, m->d.tile_off, m->d.pair_r,
-                                         m->d.pair_j, stream);
-        if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    auto* table = al.temp<unsigned long long>(slots * 2);
+    uint32_t* keys[2] = {nullptr, nullptr};
+    int32_t* vals[2] = {nullptr, nullptr};
+    uint32_t* hist = nullptr;
+    if (k3) {
+        d.nbr = al.get<int32_t>((size_t)n * spconv::kVol3, m->owned);
+        d.perm = al.get<int32_t>((size_t)n, m->owned);
+        d.nbr_t = al.get<int32_t>((size_t)d.npad * spconv::kVol3, m->owned);
+        d.win_jobs = al.get<uint32_t>((size_t)d.win_tiles * spconv::kWinJobStride, m->owned);
+        d.idx_off = al.get<int64_t>((size_t)d.win_tiles + 1, m->owned);
+        d.win_order = al.get<int32_t>((size_t)d.win_tiles, m->owned);
+        // a tile's stream holds at most its rows for each of the 27 offsets
+        d.idx_stream = al.get<int32_t>((size_t)d.npad * spconv::kVol3, m->owned);
+        keys[0] = al.temp<uint32_t>((size_t)n);
+        keys[1] = al.temp<uint32_t>((size_t)n);
+        vals[1] = al.temp<int32_t>((size_t)n);
+        vals[0] = al.temp<int32_t>((size_t)n);
+        hist = al.temp<uint32_t>((size_t)spconv::radix_hist_words(n));
     }
+    e = al.err;
+    if (e == cudaSuccess) e = cudaMemsetAsync(d.fwd_err, 0, sizeof(unsigned int), stream);
+    if (e == cudaSuccess)
+        e = spconv::launch_build_map(coords, n, extent, kernel_size, table, slots, d.nbr, keys[0], flags, stream);
+    if (e == cudaSuccess && k3) {
+        // rows sorted by the Gray rank of their neighbour mask (26 bits); the
+        // first pass takes the row indices as values
+        int which = 0;
+        e = spconv::radix_sort_pairs(keys, nullptr, vals, n, 26, hist, &which, stream);
+        if (e == cudaSuccess)
+            e = spconv::launch_win_meta(d.nbr, vals[which], n, d.win_rows, d.win_tiles, d.npad, d.perm, d.nbr_t,
+                                        d.win_jobs, d.idx_off, d.idx_stream, flags, stream);
+        // the tile claim order: tiles sorted (stably) by descending estimated cost;
+        // the row sort's buffers are free again and hold at least `tiles` entries
+        if (e == cudaSuccess) e = spconv::launch_win_cost(d.win_jobs, d.win_tiles, keys[0], stream);
+        int which_t = 0;
+        if (e == cudaSuccess) e = spconv::radix_sort_pairs(keys, nullptr, vals, d.win_tiles, 16, hist, &which_t, stream);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(d.win_order, vals[which_t], (size_t)d.win_tiles * sizeof(int32_t),
+                                cudaMemcpyDeviceToDevice, stream);
+    }
+    if (e == cudaSuccess) e = cudaMemcpyAsync(&host_flags, flags, sizeof(host_flags), cudaMemcpyDeviceToHost, stream);
+    al.release_scratch();
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    spconv_status_t status = SPCONV_OK;
     if (e != cudaSuccess) {
         status = fail_cuda(e, "spconv_build_map");
     } else if (host_flags.err & spconv::kErrCoordRange) {
@@ -131,27 +242,18 @@ spconv_status_t spconv_build_map(const int32_t* coords, int64_t n, const int32_t
         status = fail(SPCONV_ERR_DUPLICATE, "duplicate (b, x, y, z) coordinates");
     } else if (host_flags.err & spconv::kErrTableFull) {
         status = fail(SPCONV_ERR_TABLE_FULL, "hash table full");
+    } else if (host_flags.err & spconv::kErrInternal) {
+        status = fail(SPCONV_ERR_CUDA, "internal error: a metadata bound did not hold");
     }
-    cudaFree(table);
-    cudaFree(flags);
     if (status != SPCONV_OK) {
         spconv_free(m);
         return status;
     }
-    m->d.pairs = kernel_size == 3 ? (int64_t)host_flags.pairs : n;
+    d.pairs = kernel_size == 3 ? (int64_t)host_flags.pairs : n;
+    d.win_spans = (int64_t)host_flags.spans;
+    d.win_span_cols = (int64_t)host_flags.span_cols;
+    d.max_tile_cols = (int64_t)host_flags.max_tile_cols;
     *out_map = m;
-    return SPCONV_OK;
-}
-
-spconv_status_t spconv_free(spconv_map_t map) {
-    if (!map) return SPCONV_OK;
-    cudaFree(map->d.nbr);
-    cudaFree(map->d.fwd_err);
-    cudaFree(map->d.tile_counts);
-    cudaFree(map->d.tile_off);
-    cudaFree(map->d.pair_r);
-    cudaFree(map->d.pair_j);
-    delete map;
     return SPCONV_OK;
 }
 
@@ -162,6 +264,20 @@ spconv_status_t spconv_map_info(spconv_map_t map, int64_t* n, int32_t* kernel_si
     if (kernel_size) *kernel_size = map->d.kernel_size;
     if (pairs) *pairs = map->d.pairs;
     if (nbr_dev) *nbr_dev = map->d.nbr;
+    return SPCONV_OK;
+}
+
+spconv_status_t spconv_map_stats(spconv_map_t map, spconv_map_stats_t* stats) {
+    if (!map || !stats) return fail(SPCONV_ERR_INVALID_ARG, "null map or stats");
+    stats->tiles = map->d.win_tiles;
+    stats->rows_per_tile = map->d.win_rows;
+    stats->spans = map->d.win_spans;
+    stats->span_cols = map->d.win_span_cols;
+    stats->perm_dev = map->d.perm;
+    stats->nbr_t_dev = map->d.nbr_t;
+    stats->jobs_dev = map->d.win_jobs;
+    stats->job_stride = spconv::kWinJobStride;
+    stats->order_dev = map->d.win_order;
     return SPCONV_OK;
 }
 
@@ -209,25 +325,34 @@ spconv_status_t spconv_subm_forward_algo(spconv_map_t map, spconv_dtype_t dtype,
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
     if (algo == SPCONV_ALGO_TCGEN05 && dtype != SPCONV_BF16)
         return fail(SPCONV_ERR_UNSUPPORTED, "the tcgen05 kernel is bf16 only");
-    if (dtype == SPCONV_BF16 && algo != SPCONV_ALGO_SIMT) {
+    // AUTO: bf16 with cout % 64 == 0 runs on the tensor cores; fp32 and other bf16
+    // shapes on the CUDA-core kernel.  The choice depends on the shape alone, and
+    // the map's launch counters record it.
+    const bool tc_shape = dtype == SPCONV_BF16 && cout % 64 == 0;
+    if (algo == SPCONV_ALGO_TCGEN05 || (algo == SPCONV_ALGO_AUTO && tc_shape)) {
         cudaError_t ce = cudaSuccess;
-        spconv_status_t s = spconv::launch_forward_tcgen05(map->d, x, cin, w, bias, out, cout, stream, &ce);
+        const spconv_status_t s = spconv::launch_forward_tcgen05(map->d, x, cin, w, bias, out, cout, stream, &ce);
         if (s == SPCONV_ERR_CUDA) return fail_cuda(ce, "tcgen05 forward");
-        if (s == SPCONV_OK) return SPCONV_OK;
-        // The tensor-core kernel takes cout % 64 == 0; AUTO runs other bf16 shapes
-        // on the CUDA-core kernel.
-        if (algo == SPCONV_ALGO_TCGEN05)
-            return fail(s, "tcgen05 forward does not take this shape (cout % 64 != 0, cin % 16 != 0, or the tile lists "
-                           "do not fit shared memory)");
+        if (s != SPCONV_OK)
+            return fail(s, "the tcgen05 kernel does not take this shape (bf16 with cout % 64 == 0 and cin % 16 == 0)");
+        map->launches[SPCONV_KERNEL_TCGEN05].fetch_add(1);
+        return SPCONV_OK;
     }
     cudaError_t e = spconv::launch_forward_simt(map->d, dtype, x, cin, w, bias, out, cout, stream);
     if (e != cudaSuccess) return fail_cuda(e, "simt forward");
+    map->launches[SPCONV_KERNEL_SIMT].fetch_add(1);
     return SPCONV_OK;
 }
 
 spconv_status_t spconv_subm_forward(spconv_map_t map, spconv_dtype_t dtype, const void* x, int32_t cin,
                                     const void* w, const void* bias, void* out, int32_t cout, void* stream) {
     return spconv_subm_forward_algo(map, dtype, x, cin, w, bias, out, cout, SPCONV_ALGO_AUTO, stream);
+}
+
+spconv_status_t spconv_map_launch_counts(spconv_map_t map, int64_t* counts, int32_t ncounts) {
+    if (!map || !counts || ncounts < 1) return fail(SPCONV_ERR_INVALID_ARG, "null map or counts, or ncounts < 1");
+    for (int32_t k = 0; k < ncounts; ++k) counts[k] = k < SPCONV_KERNEL_KINDS ? map->launches[k].load() : 0;
+    return SPCONV_OK;
 }
 
 }  // extern "C"

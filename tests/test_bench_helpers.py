@@ -86,19 +86,19 @@ def test_kernel_source_hash_ignores_comments_but_not_code(tmp_path, monkeypatch)
         shutil.copy(os.path.join(ROOT, "submanifold_sparse_convolution_submconv3d_b200", "csrc", name), csrc / name)
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     h0 = bench.kernel_sources_sha256()
-    f = csrc / "forward_tc.cu"
+    f = csrc / "forward_win.cu"
     src = f.read_text()
     f.write_text("// a new comment line\n" + src.replace("\n", "  \n", 3) + "\n/* trailing\n block */\n")
     assert bench.kernel_sources_sha256() == h0
-    f.write_text(src.replace("kJobRows = 48", "kJobRows = 32", 1))
+    f.write_text(src.replace("kUnitRows = 64", "kUnitRows = 32", 1))
     assert bench.kernel_sources_sha256() != h0
 
 
 def test_tc_kernel_name_follows_the_dispatch():
-    assert bench.tc_kernel_name(128, 128) == "k_subm_tc<128,128>"
-    assert bench.tc_kernel_name(64, 64) == "k_subm_tc<64,64>"
-    assert bench.tc_kernel_name(48, 192) == "k_subm_tc<64,16>"
-    assert bench.tc_kernel_name(32, 256) == "k_subm_tc<128,32>"
+    assert bench.tc_kernel_name(128, 128) == "k_subm_win<128,128>"
+    assert bench.tc_kernel_name(64, 64) == "k_subm_win<64,64>"
+    assert bench.tc_kernel_name(48, 192) == "k_subm_win<64,16>"
+    assert bench.tc_kernel_name(32, 256) == "k_subm_win<128,32>"
 
 
 def test_column_efficiency_of_the_bench_workload():

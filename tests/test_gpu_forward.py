@@ -1,8 +1,10 @@
 """GPU forward vs the CPU oracle (fp64), through the C ABI.
 
-Small cases are compared on every output row; the full-size workloads are
-compared on sampled rows the oracle computes one by one (the RMS in the
-tolerance is then taken over the sampled reference rows).
+Every comparison takes its reference from the oracle alone: the oracle's own
+neighbour map and the oracle's forward, never a map or value from the CUDA path.
+Small cases and the full-size workloads are compared on every output row (the
+oracle runs on row chunks in parallel host threads); the ten chained layers of
+the 128^3 workload are compared on sampled rows per layer, beside one full layer.
 """
 import numpy as np
 import pytest
@@ -10,7 +12,7 @@ import torch
 
 import oracle
 import workloads
-from gpu_helpers import assert_close, coords_dev, to_dev
+from gpu_helpers import assert_close, coords_dev, oracle_forward_rows, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -121,10 +123,10 @@ def tile_rows(sp):
     sp.spconv_debug_set_tile_rows(0)
 
 
-# Small inputs get short automatic tiles; the same cases through full-height
-# (384-row) tiles and an odd height exercise several jobs per offset, every
-# centre job of a tile and ragged tails inside a tile.
-@pytest.mark.parametrize("rows", [384, 100])
+# The same cases through full-height (256-row) tiles, the shortest (16-row) tiles
+# and an odd number of windows per tile: spans of every length, many tiles per
+# CTA (both accumulator buffers, several rounds each) and ragged tails.
+@pytest.mark.parametrize("rows", [256, 16, 112])
 @pytest.mark.parametrize("cin,cout,kvol", [(128, 128, 27), (64, 128, 27), (16, 64, 27), (512, 512, 27),
                                            (128, 128, 1), (48, 128, 1)])
 def test_bf16_tcgen05_forced_tile_heights(sp, tile_rows, rows, cin, cout, kvol):
@@ -136,7 +138,7 @@ def test_bf16_tcgen05_forced_tile_heights(sp, tile_rows, rows, cin, cout, kvol):
 
 def test_dense_block_full_height_tiles(sp, tile_rows):
     rng = np.random.default_rng(11)
-    tile_rows(384)
+    tile_rows(256)
     blk = np.array([[0, a, b, c] for a in range(12) for b in range(12) for c in range(12)], np.int32)
     blk = blk[rng.permutation(blk.shape[0])]
     x = workloads.round_to_bf16(rng.standard_normal((blk.shape[0], 128), dtype=np.float32))
@@ -147,7 +149,7 @@ def test_dense_block_full_height_tiles(sp, tile_rows):
 
 
 def test_single_voxel_and_single_tile_edge(sp):
-    for n in (1, 351, 352, 353, 383, 384, 385, 705):  # around the 384-row tile and other sizes
+    for n in (1, 15, 16, 17, 127, 128, 129, 255, 256, 257, 705):  # around windows and tile heights
         coords, ext, x, w, b = _case(6 + n, 12, n, 64, 64)
         out = _run(sp, coords, ext, x, w, b, "bf16", algo=sp.ALGO_TCGEN05)
         assert_close(out, _ref(coords, ext, x, w, b), "bf16")
@@ -172,7 +174,9 @@ def _sample_rows(n, count, seed=0):
 
 
 @pytest.mark.parametrize("name", ["shells", "batched", "large"])
-def test_full_size_workloads_sampled(sp, name):
+def test_full_size_workloads_every_row(sp, name):
+    """Every output row of the full-size workloads (batched: its k=3 layer and
+    the chained k=1 layer) against the oracle run on the same input."""
     wl = workloads.make_workload(name, 0)
     m = sp.spconv_build_map(coords_dev(wl.coords), wl.grid, 3)
     nbr = oracle.neighbor_map(wl.coords, wl.grid)
@@ -180,14 +184,13 @@ def test_full_size_workloads_sampled(sp, name):
     try:
         x_host = wl.x
         x_dev = to_dev(wl.x, "bf16")
-        for layer in wl.layers:
+        for li, layer in enumerate(wl.layers):
             mm = m if layer.kernel_size == 3 else m1
             out = sp.spconv_subm_forward(mm, x_dev, to_dev(layer.w, "bf16"), to_dev(layer.bias, "bf16"))
             mm.check()
-            rows = _sample_rows(wl.n, 1500)
             nb = nbr if layer.kernel_size == 3 else np.arange(wl.n, dtype=np.int32).reshape(-1, 1)
-            ref = oracle.forward(nb, x_host, layer.w, layer.bias, rows=rows)
-            assert_close(out[torch.from_numpy(rows).cuda()], ref, "bf16")
+            ref = oracle_forward_rows(oracle, nb, x_host, layer.w, layer.bias)
+            assert_close(out, ref, "bf16", label=f"{name} layer {li} k={layer.kernel_size}")
             if wl.chained:  # next layer consumes this layer's GPU output
                 x_dev = out
                 x_host = out.float().cpu().numpy()
@@ -228,9 +231,9 @@ def test_uniform_full_output_every_row(sp):
         tc = sp.spconv_subm_forward(m, x, w, b, algo=sp.ALGO_TCGEN05)
         simt = sp.spconv_subm_forward(m, x, w, b, algo=sp.ALGO_SIMT)
         m.check()
-        ref = oracle.forward(m.neighbor_map().cpu().numpy(), wl.x, layer.w, layer.bias)
-        assert_close(tc, ref, "bf16")
-        assert_close(simt, ref, "bf16")
+        ref = oracle_forward_rows(oracle, oracle.neighbor_map(wl.coords, wl.grid), wl.x, layer.w, layer.bias)
+        assert_close(tc, ref, "bf16", label="uniform tcgen05")
+        assert_close(simt, ref, "bf16", label="uniform simt")
     finally:
         m.free()
 
@@ -246,3 +249,43 @@ def test_repeat_calls_identical(sp):
         assert torch.equal(o1, o2)
     finally:
         m.free()
+
+
+@pytest.mark.parametrize("name", ["tiny", "uniform", "shells", "batched", "large"])
+def test_auto_kernel_choice_on_workloads(sp, name):
+    """AUTO runs every bf16 layer of the five workloads on the tensor cores (and the
+    fp32 tiny layers on the CUDA-core kernel); the map's launch counters show it."""
+    wl = workloads.make_workload(name, 0, n_layers=1)
+    expected = "simt" if wl.dtype == "f32" else "tcgen05"
+    x = to_dev(wl.x, wl.dtype)
+    for layer in wl.layers:
+        m = sp.spconv_build_map(coords_dev(wl.coords), wl.grid, layer.kernel_size)
+        try:
+            sp.spconv_subm_forward(m, x, to_dev(layer.w, wl.dtype), to_dev(layer.bias, wl.dtype))
+            m.check()
+            counts = m.launch_counts()
+        finally:
+            m.free()
+        assert counts[expected] == 1 and sum(counts.values()) == 1, (name, layer.kernel_size, counts)
+
+
+@pytest.fixture
+def ring_depths(sp):
+    """Force the forward's ring depths; restores the automatic choice."""
+    def force(a, b):
+        sp.spconv_debug_set_ring_depths(a, b)
+    yield force
+    sp.spconv_debug_set_ring_depths(0, 0)
+
+
+# Shallow rings: the weight ring and the B-ring units wrap around on nearly every
+# job (jobs that do not fit before the end start over at unit 0), including the
+# several input-channel chunks of 512-channel layers.
+@pytest.mark.parametrize("a,b", [(2, 4), (2, 5), (3, 5)])
+@pytest.mark.parametrize("cin,cout,kvol", [(128, 128, 27), (512, 512, 27), (64, 64, 27), (32, 64, 27),
+                                           (512, 512, 1)])
+def test_bf16_tcgen05_shallow_rings(sp, ring_depths, a, b, cin, cout, kvol):
+    ring_depths(a, b)
+    coords, ext, x, w, bias = _case(13, 22, 2500, cin, cout, kvol=kvol)
+    out = _run(sp, coords, ext, x, w, bias, "bf16", algo=sp.ALGO_TCGEN05)
+    assert_close(out, _ref(coords, ext, x, w, bias), "bf16", label=f"rings {a},{b}")

@@ -96,16 +96,112 @@ def test_map_errors(sp):
     _check_map(sp, coords, (16, 16, 16))
 
 
-def test_tile_height_fills_whole_waves(sp):
-    """The map picks the smallest tile that keeps the wave count 384-row tiles need."""
-    import torch
+@pytest.mark.parametrize("name", ["uniform", "shells", "large"])
+def test_tile_height_balances_the_sms(sp, name):
+    """The map's tile height is a multiple of 16 in [128, 256], and no other such
+    height gives the busiest SM fewer rows when the tiles are dealt out round-robin
+    over the device's SMs."""
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    wl = workloads.make_workload("uniform", 0, n_layers=1)
+    wl = workloads.make_workload(name, 0, n_layers=1)
     m = sp.spconv_build_map(coords_dev(wl.coords), wl.grid, 3)
     try:
         rows, n = m.tile_rows, wl.n
-        waves = -(-n // (384 * sms))
-        assert rows <= 384 and -(-n // rows) <= waves * sms
-        assert rows == 384 or -(-n // (rows - 1)) > waves * sms
     finally:
         m.free()
+
+    def busiest(r):
+        return -(-(-(-n // r)) // sms) * r
+
+    assert rows % 16 == 0 and 128 <= rows <= 256
+    assert all(busiest(rows) <= busiest(r) for r in range(128, 257, 16))
+
+
+# ---------------------------------------------------------------------------
+# The tensor-core forward's metadata, against a host derivation from the oracle's
+# map: the row order is fully determined (a stable sort by the Gray-code rank of
+# the 26-bit neighbour mask), so it and the permuted table compare bit for bit;
+# the spans are a cost-model choice, so they are checked for what any valid cover
+# must satisfy.
+
+def _gray_rank(v: np.ndarray) -> np.ndarray:
+    r = v.copy()
+    s = v >> 1
+    while s.any():
+        r ^= s
+        s >>= 1
+    return r
+
+
+def _expected_order(nbr: np.ndarray) -> np.ndarray:
+    nc = np.delete(nbr >= 0, 13, axis=1)
+    key = nc.astype(np.int64) @ (1 << np.arange(25, -1, -1)).astype(np.int64)
+    return np.argsort(_gray_rank(key), kind="stable")
+
+
+def _check_window_meta(sp, coords, extent):
+    m = sp.spconv_build_map(coords_dev(coords), extent, 3)
+    try:
+        st = m.stats(copy_arrays=True)
+    finally:
+        m.free()
+    ref = oracle.neighbor_map(coords, extent)
+    n = ref.shape[0]
+    rows, tiles = st["rows_per_tile"], st["tiles"]
+    assert rows % 16 == 0 and 16 <= rows <= 256 and tiles == -(-n // rows)
+    perm = st["perm"].cpu().numpy()
+    assert np.array_equal(perm, _expected_order(ref))
+    npad = rows * tiles
+    exp_t = np.full((27, npad), -1, np.int32)
+    exp_t[:, :n] = ref[perm].T
+    assert np.array_equal(st["nbr_t"].cpu().numpy(), exp_t)
+    jobs = st["jobs"].cpu().numpy()
+    nwin = rows // 16
+    occ = (exp_t.reshape(27, tiles, nwin, 16) >= 0).any(axis=3)  # [27, tiles, windows]
+    spans = cols = 0
+    stream_start = 0
+    for t in range(tiles):
+        nj = int(jobs[t, 0])
+        js = jobs[t, 4:4 + nj]
+        # header: the tile's index stream length and start (tiles' streams are consecutive)
+        assert int(jobs[t, 2]) | (int(jobs[t, 3]) << 32) == stream_start
+        assert int(jobs[t, 1]) == int(((js >> 16) & 31).sum()) * 16
+        stream_start += int(jobs[t, 1])
+        k, w0, nw = js & 31, (js >> 8) & 31, (js >> 16) & 31
+        assert (k[0], w0[0], nw[0]) == (13, 0, nwin)  # the centre job covers the tile
+        k, w0, nw = k[1:], w0[1:], nw[1:]
+        assert np.all(k != 13) and np.all(k < 27) and np.all(nw >= 1) and np.all(w0 + nw <= nwin)
+        # each offset's spans are listed together, in increasing window order, without overlap
+        runs = k[np.r_[True, k[1:] != k[:-1]]] if k.size else k
+        assert len(runs) == len(set(runs.tolist()))
+        cover = np.zeros((27, nwin), np.int32)
+        for kk, a, b in zip(k, w0, nw):
+            cover[kk, a:a + b] += 1
+        assert cover.max(initial=0) <= 1
+        need = occ[:, t, :].copy()
+        need[13] = False
+        assert np.all(cover[need] == 1), f"tile {t}: a window with a neighbour is not covered"
+        spans += len(k)
+        cols += int(nw.sum()) * 16
+    assert spans == st["spans"] and cols == st["span_cols"]
+    # claim order: a stable sort of the tiles by descending cost 4 * J + stream length // 16
+    cost = np.minimum(4 * jobs[:, 0] + jobs[:, 1] // 16, 0xFFFF)
+    order = st["order"].cpu().numpy()
+    assert np.array_equal(order, np.argsort(-cost, kind="stable"))
+
+
+@pytest.mark.parametrize("name", ["tiny", "uniform", "shells", "batched", "large"])
+def test_window_metadata_on_workloads(sp, name):
+    wl = workloads.make_workload(name, 0, n_layers=1)
+    _check_window_meta(sp, wl.coords, wl.grid)
+
+
+@pytest.mark.parametrize("rows", [16, 256, 112])
+def test_window_metadata_forced_tile_heights(sp, rows):
+    sp.spconv_debug_set_tile_rows(rows)
+    try:
+        rng = np.random.default_rng(rows)
+        _check_window_meta(sp, workloads.uniform_coords(rng, 24, 3000), (24, 24, 24))
+        blk = np.array([[0, a, b, c] for a in range(10) for b in range(10) for c in range(10)], np.int32)
+        _check_window_meta(sp, blk[rng.permutation(1000)], (10, 10, 10))
+    finally:
+        sp.spconv_debug_set_tile_rows(0)

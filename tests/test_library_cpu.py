@@ -64,9 +64,19 @@ def test_host_validation_without_device_work(pkg):
     rows = ctypes.c_int32()
     assert lib.spconv_map_tile_rows(None, ctypes.byref(rows)) == pkg.INVALID_ARG
     assert lib.spconv_debug_set_tile_rows(-1) == pkg.INVALID_ARG
-    assert lib.spconv_debug_set_tile_rows(385) == pkg.INVALID_ARG
-    assert lib.spconv_debug_set_tile_rows(384) == pkg.OK
+    assert lib.spconv_debug_set_tile_rows(272) == pkg.INVALID_ARG
+    assert lib.spconv_debug_set_tile_rows(100) == pkg.INVALID_ARG  # not a multiple of 16
+    assert lib.spconv_debug_set_tile_rows(256) == pkg.OK
+    assert lib.spconv_debug_set_tile_rows(16) == pkg.OK
     assert lib.spconv_debug_set_tile_rows(0) == pkg.OK
+    assert lib.spconv_debug_set_ring_depths(1, 8) == pkg.INVALID_ARG
+    assert lib.spconv_debug_set_ring_depths(3, 3) == pkg.INVALID_ARG
+    assert lib.spconv_debug_set_ring_depths(3, 33) == pkg.INVALID_ARG
+    assert lib.spconv_debug_set_ring_depths(2, 4) == pkg.OK
+    assert lib.spconv_debug_set_ring_depths(0, 0) == pkg.OK
+    assert lib.spconv_map_stats(None, None) == pkg.INVALID_ARG
+    counts = (ctypes.c_int64 * 2)()
+    assert lib.spconv_map_launch_counts(None, counts, 2) == pkg.INVALID_ARG
 
 
 def test_python_binding_rejects_bad_tensors(pkg):
