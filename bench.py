@@ -3,12 +3,17 @@ occupancy, plus map-build ms (the workload of the lato.2_mrp_mlx README's
 "Fleet benchmark": 209,715 voxels, 128 -> 128 channels, warm neighbour map).
 
 One step = ten chained 128 -> 128 bf16 layers over one cached map (ping-pong
-buffers), inputs resident in HBM; value = active voxels x layers / step seconds
-/ 1e6 (Mvox/s per layer, the pages' unit).  L2 is flushed (a 512 MB write)
-between timed steps; each step is timed with CUDA events on the launching stream.
-The map build is timed separately (map_build_ms).  e2e repeats the step through
-the public API from pinned host buffers: coordinates, features and weights
-copied in, map built, ten layers, output copied back.
+buffers), inputs resident in HBM, launched as one captured CUDA graph; value =
+active voxels x layers / step seconds / 1e6 (Mvox/s per layer, the pages' unit).
+L2 is flushed (a 512 MB write) before every timed step; each step is timed with
+CUDA events on the launching stream.  The map build is timed separately
+(map_build_ms).  e2e repeats the step through the public API from pinned host
+buffers: coordinates, features and weights copied in, map built, ten layers,
+output copied back.
+
+per_config times the other workloads' layers the same way (one captured layer,
+L2 flushed before each replay), each against its own roofline, and the 512^3
+shell workload end to end (map build + layer).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -47,11 +52,17 @@ CONFIG = {
     "workload": "SubMConv3d k=3, 128^3 grid, 209,715 active voxels (~10%) uniform without replacement, "
                 "batch 1, 128->128 channels, bf16 in / fp32 accumulate, map built once and reused for 10 layers",
     "grid": 128, "voxels": 209715, "cin": 128, "cout": 128, "kernel_size": 3, "layers_per_step": LAYERS,
-    "l2": "flushed between timed steps (512 MB write)",
+    "l2": "flushed before every timed step (512 MB write)",
+    "launch": "each step is one captured CUDA graph of the ten layers",
 }
+PER_CONFIG = (  # (workload, layer index, label)
+    ("shells", 0, "shells k=3 64->64"),
+    ("batched", 0, "batched k=3 512->512"),
+    ("batched", 1, "batched k=1 512->512"),
+    ("large", 0, "large k=3 32->64"),
+)
 
-
-# DRAM traffic of one forward launch from the committed ncu capture
+# DRAM traffic of one forward launch from a committed ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
 # sources it was taken on: reported as null once their hash changes.
 PROFILED_TRAFFIC = {
@@ -164,75 +175,174 @@ def whole_job_mvox(world: int, steps: int, layers: int, n: int, total_ms: float)
     return world * steps * layers * n / (total_ms / 1e3) / 1e6
 
 
-def mma_column_efficiency(nbr: np.ndarray, tile_rows: int, bm: int = 128, job_rows: int = 48,
-                          n_align: int = 16) -> float:
-    """Fraction of the MMA columns the forward issues that carry a real pair.
-
-    Per tile it issues centre jobs of bm rows and, per other offset, jobs of up to
-    job_rows compacted hits; each job's MMA N is rounded up to n_align."""
-    n = nbr.shape[0]
-    t = -(-n // tile_rows)
-    hits = np.zeros((t * tile_rows, nbr.shape[1]), dtype=bool)
-    hits[:n] = nbr >= 0
-    counts = hits.reshape(t, tile_rows, -1).sum(axis=1)  # [tiles, 27]
-
-    def issued(c: np.ndarray, chunk: int) -> int:
-        rem = c % chunk
-        return int((c // chunk).sum() * chunk + ((rem + n_align - 1) // n_align * n_align).sum())
-
-    centre = nbr.shape[1] // 2
-    cols = issued(counts[:, centre], bm)
-    for k in range(nbr.shape[1]):
-        if k != centre:
-            cols += issued(counts[:, k], job_rows)
-    return float(hits.sum()) / cols
+def issued_column_efficiency(pairs: int, npad: int, span_cols: int) -> float:
+    """Fraction of the MMA columns the forward issues that carry a (voxel, offset)
+    pair: every tile's centre job issues one column per tile row (npad in all,
+    padding rows of the last tile included) and the spans issue span_cols more."""
+    issued = npad + span_cols
+    return float(pairs) / issued if issued else 1.0
 
 
-def roofline_bytes_flops(n: int, pairs: int, cin: int, cout: int) -> tuple[float, float]:
-    """Compulsory bytes and useful FLOPs of one k=3 layer: x read once, W once, bias,
+def roofline_bytes_flops(n: int, pairs: int, cin: int, cout: int, kvol: int = 27) -> tuple[float, float]:
+    """Compulsory bytes and useful FLOPs of one layer: x read once, W once, bias,
     out written once, 4 bytes per non-centre neighbour pair; 2*Cin*Cout per pair."""
-    byts = n * cin * 2 + 27 * cin * cout * 2 + cout * 2 + n * cout * 2 + 4 * (pairs - n)
+    byts = n * cin * 2 + kvol * cin * cout * 2 + cout * 2 + n * cout * 2 + 4 * (pairs - n)
     flops = 2.0 * cin * cout * pairs
     return float(byts), flops
 
 
-def cpu_baseline(wl, target_s: float = 10.0) -> dict:
-    """The CPU oracle (plain C, fp64, one thread), as it stands, on a bounded sample:
-    the full neighbour map, then the first layer's forward on a row sample sized for
-    about target_s seconds.  Returns Mvox/s per layer = sampled rows / forward seconds."""
+def roofline(n: int, pairs: int, cin: int, cout: int, kvol: int, layer_s: float, hbm_gbs: float,
+             tflops: float) -> dict:
+    """The layer against the slower of its compulsory bytes at HBM bandwidth and its
+    useful FLOPs at the bf16 tensor peak."""
+    byts, flops = roofline_bytes_flops(n, pairs, cin, cout, kvol)
+    t_hbm, t_tensor = byts / (hbm_gbs * 1e9), flops / (tflops * 1e12)
+    bound = "hbm" if t_hbm >= t_tensor else "tensor"
+    return {"bound": bound, "t_roof_us": max(t_hbm, t_tensor) * 1e6, "frac": max(t_hbm, t_tensor) / layer_s,
+            "achieved_gbs": byts / layer_s / 1e9, "achieved_tflops": flops / layer_s / 1e12,
+            "algorithmic_bytes": byts, "useful_flops": flops}
+
+def capture_graph(fn):
+    """Run fn twice on a side stream (first launches set up the library), then
+    capture one call of it into a CUDA graph."""
+    import torch
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for _ in range(2):
+            fn()
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g
+
+
+def time_replays(g, reps: int, flush, before=None) -> list[float]:
+    """CUDA-event times (ms) of `reps` replays of graph g on the current stream, L2
+    flushed (and `before` run) ahead of each replay, outside the timed interval."""
+    import torch
+    out = []
+    stream = torch.cuda.current_stream()
+    for _ in range(reps):
+        if before is not None:
+            before()
+        flush.fill_(1.0)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        out.append(e0.elapsed_time(e1))
+    return out
+
+
+def cpu_oracle_sample(wl, layer, target_s: float) -> dict:
+    """The CPU oracle (plain C, fp64, one thread), as it stands, on a bounded sample
+    of one layer: the full neighbour map, then the forward on the first rows, as many
+    as take about target_s seconds.  Mvox/s = sampled rows / forward seconds: an
+    extrapolation to the whole layer at the sampled rate."""
     import oracle
     t0 = time.perf_counter()
-    nbr = oracle.neighbor_map(wl.coords, wl.grid)
+    nbr = oracle.neighbor_map(wl.coords, wl.grid, layer.kernel_size)
     build_s = time.perf_counter() - t0
-    layer = wl.layers[0]
-    probe = np.arange(0, min(wl.n, 2000))
+    probe = np.arange(0, min(wl.n, 500))
     t0 = time.perf_counter()
     oracle.forward(nbr, wl.x, layer.w, layer.bias, rows=probe)
     per_row = max((time.perf_counter() - t0) / len(probe), 1e-9)
-    rows = np.arange(0, int(min(wl.n, max(2000, target_s / per_row))))
+    rows = np.arange(0, int(min(wl.n, max(500, target_s / per_row))))
     t0 = time.perf_counter()
     oracle.forward(nbr, wl.x, layer.w, layer.bias, rows=rows)
     fwd_s = time.perf_counter() - t0
-    return {"value": len(rows) / fwd_s / 1e6, "unit": UNIT, "cores": 1, "kind": "oracle",
+    return {"value": len(rows) / fwd_s / 1e6, "unit": UNIT, "cores": 1, "kind": "oracle", "extrapolated": len(rows) < wl.n,
+            "rows_timed": int(len(rows)), "rows_total": int(wl.n), "seconds_timed": round(fwd_s, 3),
+            "map_build_s": round(build_s, 3),
             "sample": f"C oracle (fp64, 1 thread): neighbour map of all {wl.n} voxels in {build_s * 1e3:.0f} ms, "
-                      f"then layer 1 forward on the first {len(rows)} of {wl.n} rows in {fwd_s:.2f} s"}
+                      f"then the forward of the first {len(rows)} of {wl.n} rows in {fwd_s:.2f} s"}
 
+
+def run_per_config(sp, dev, flush, reps: int, hbm: float, tflops: float, cpu: bool) -> list[dict]:
+    """One layer of each other workload (captured, L2 flushed before each replay)
+    against its roofline; the 512^3 shells also end to end (map build + layer)."""
+    import torch
+    results = []
+    cache = {}
+    for name, li, label in PER_CONFIG:
+        wl = cache.setdefault(name, workloads.make_workload(name, 0))
+        layer = wl.layers[li]
+        ks = layer.kernel_size
+        kvol, cin, cout = layer.w.shape
+        coords_d = torch.from_numpy(wl.coords).to(dev)
+        m = sp.spconv_build_map(coords_d, wl.grid, ks)
+        x = torch.from_numpy(wl.x).to(dev, torch.bfloat16)
+        w = torch.from_numpy(layer.w).to(dev, torch.bfloat16)
+        b = torch.from_numpy(layer.bias).to(dev, torch.bfloat16)
+        o = torch.empty((wl.n, cout), dtype=torch.bfloat16, device=dev)
+        g = capture_graph(lambda: sp.spconv_subm_forward(m, x, w, b, out=o))
+        for _ in range(3):
+            g.replay()
+        ms = time_replays(g, reps, flush)
+        m.check()
+        layer_s = statistics.median(ms) / 1e3
+        st = m.stats()
+        e = {"config": label, "workload": name, "voxels": wl.n, "pairs": m.pairs, "cin": int(cin), "cout": int(cout),
+             "kernel_size": ks, "layer_us_median": layer_s * 1e6, "layer_us_min": min(ms) * 1e3,
+             "mvox_s": wl.n / layer_s / 1e6, "kernel": tc_kernel_name(int(cin), int(cout)),
+             "roofline": roofline(wl.n, m.pairs, int(cin), int(cout), int(kvol), layer_s, hbm, tflops),
+             "rows_per_tile": st["rows_per_tile"], "tiles": st["tiles"], "launch_counts": m.launch_counts()}
+        if ks == 3:
+            e["spans"] = st["spans"]
+            e["issued_column_efficiency"] = issued_column_efficiency(m.pairs, st["tiles"] * st["rows_per_tile"],
+                                                                     st["span_cols"])
+        del g
+        m.free()
+        if name == "large":
+            # end to end on the GPU: map build (hash, probe, row sort, tile metadata;
+            # one stream synchronisation inside) then the layer, host-timed
+            e2e, builds, fwds = [], [], []
+            for _ in range(4):
+                flush.fill_(1.0)
+                torch.cuda.synchronize()
+                t0 = time.perf_counter()
+                mm = sp.spconv_build_map(coords_d, wl.grid, 3)
+                t1 = time.perf_counter()
+                sp.spconv_subm_forward(mm, x, w, b, out=o)
+                torch.cuda.synchronize()
+                t2 = time.perf_counter()
+                mm.free()
+                e2e.append((t2 - t0) * 1e3)
+                builds.append((t1 - t0) * 1e3)
+                fwds.append((t2 - t1) * 1e3)
+            e["end_to_end"] = {"ms_median": statistics.median(e2e[1:]), "map_build_ms_median": statistics.median(builds[1:]),
+                               "forward_ms_median": statistics.median(fwds[1:]),
+                               "includes": "map build (one stream synchronisation) + one layer, host-timed, L2 flushed"}
+        if cpu:
+            e["cpu_baseline"] = cpu_oracle_sample(wl, layer, target_s=1.5)
+        results.append(e)
+        del x, w, b, o, coords_d
+        torch.cuda.empty_cache()
+    return results
 
 def run_reference(args, rank: int, world: int) -> None:
+    """The reference arm: the CPU oracle as it stands on the host cores (rank 0 only),
+    each step a bounded sample of the headline layer; the per-layer rate is an
+    extrapolation from the sampled rows and is marked as such."""
     if rank != 0:
         return
     wl = workloads.make_workload(WORKLOAD, 0, n_layers=1)
     per_step = []
     base = None
     for i in range(args.warmup + args.steps):
-        b = cpu_baseline(wl, target_s=max(2.0, min(10.0, 60.0 / max(1, args.steps + args.warmup))))
+        b = cpu_oracle_sample(wl, wl.layers[0], target_s=max(1.0, min(10.0, 60.0 / max(1, args.steps + args.warmup))))
         if i >= args.warmup:
             per_step.append(b["value"])
             base = b
     value = statistics.median(per_step)
     base["value"] = value
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": LAYERS * wl.n / (value * 1e6) * 1e3,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": LAYERS * wl.n / (value * 1e6) * 1e3,
+            "ms_per_step_extrapolated": True,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": value / PAGES_MVOX, "vs_baseline_ref": PAGES_REF,
             "dtype": "f64", "data": "synthetic",
             "config": CONFIG, "cpu_baseline": base,
@@ -267,50 +377,38 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
 
     m = sp.spconv_build_map(coords_d, wl.grid, 3)
     pairs = m.pairs
-    col_eff = mma_column_efficiency(m.neighbor_map().cpu().numpy(), m.tile_rows)
+    st = m.stats()
 
-    def step(events=None):
+    def step():
         for i in range(LAYERS):
-            src, dst = bufs[i % 2], bufs[(i + 1) % 2]
-            if events is not None:
-                events[i][0].record(stream)
-            sp.spconv_subm_forward(m, src, ws[i], bs[i], out=dst)
-            if events is not None:
-                events[i][1].record(stream)
+            sp.spconv_subm_forward(m, bufs[i % 2], ws[i], bs[i], out=bufs[(i + 1) % 2])
+
+    graph = capture_graph(step)
+    for _ in range(args.warmup):
+        bufs[0].copy_(x0)
+        graph.replay()
+    m.check()
 
     def barrier():
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
 
-    for _ in range(args.warmup):
-        bufs[0].copy_(x0)
-        step()
-    m.check()
-
-    # ---- timed region: K steps, L2 flushed between them
+    # ---- timed region: K steps (one graph replay each), L2 flushed before each
     visible = [s for s in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if s]
     sampler = ClockSampler(visible[local_rank] if local_rank < len(visible) else str(local_rank))
     sampler.start()
-    layer_ms, step_ms = [], []
     barrier()
-    for _ in range(args.steps):
-        bufs[0].copy_(x0)
-        flush.fill_(1.0)
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(LAYERS)]
-        step(ev)
-        torch.cuda.synchronize()
-        ms = [a.elapsed_time(b) for a, b in ev]
-        layer_ms.extend(ms)
-        step_ms.append(ev[0][0].elapsed_time(ev[-1][1]))
+    step_ms = time_replays(graph, args.steps, flush, before=lambda: bufs[0].copy_(x0))
     barrier()
     clocks = sampler.stop()
     m.check()
-    total_ms = sum(step_ms)
-    total_ms = max_over_ranks(total_ms, world, dev)
+    counts = m.launch_counts()
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
     value = whole_job_mvox(world, args.steps, LAYERS, n, total_ms)
 
-    # ---- map build, timed separately (pack + insert + probe, one host sync inside)
+    # ---- map build, timed separately (pack + insert + probe + row sort + tile
+    # metadata, one stream synchronisation inside)
     build_ms = []
     for i in range(max(3, args.steps)):
         flush.fill_(1.0)
@@ -320,7 +418,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         build_ms.append((time.perf_counter() - t0) * 1e3)
         mm.free()
 
-    # ---- e2e through the public API from pinned host memory
+    # ---- e2e through the public API from pinned host memory (no graph)
     h2d = coords_h.numel() * 4 + x_h.numel() * 2 + sum(w.numel() * 2 for w in w_h) + sum(b.numel() * 2 for b in b_h)
     d2h = out_h.numel() * 2
     e2e_ms = []
@@ -343,48 +441,57 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         me.free()
         if i >= args.warmup:
             e2e_ms.append(dt)
-    e2e_total = sum(e2e_ms)
-    e2e_total = max_over_ranks(e2e_total, world, dev)
+    e2e_total = max_over_ranks(sum(e2e_ms), world, dev)
     e2e_value = whole_job_mvox(world, args.steps, LAYERS, n, e2e_total)
 
+    hbm, tf_burst, tf_sust, peak_kind = _peaks()
+    layer_s = statistics.median(step_ms) / LAYERS / 1e3
+    per_config = None
+    if world == 1 and not args.no_per_config:
+        per_config = run_per_config(sp, dev, flush, 10, hbm, tf_burst, cpu=not args.no_cpu_baseline)
     if rank != 0:
         return
-    hbm, tf_burst, tf_sust, peak_kind = _peaks()
-    byts, flops = roofline_bytes_flops(n, pairs, cin, cout)
-    avg_launch_s = statistics.mean(layer_ms) / 1e3
-    achieved_gbs = byts / avg_launch_s / 1e9
-    t_hbm, t_tensor = byts / (hbm * 1e9), flops / (tf_burst * 1e12)
+    rf = roofline(n, pairs, cin, cout, 27, layer_s, hbm, tf_burst)
     kname = tc_kernel_name(cin, cout)
     traffic = None
-    if kname == PROFILED_TRAFFIC["kernel"] and kernel_sources_sha256() == PROFILED_TRAFFIC["sources_sha256"]:
+    if (PROFILED_TRAFFIC["bytes"] is not None and kname == PROFILED_TRAFFIC["kernel"]
+            and kernel_sources_sha256() == PROFILED_TRAFFIC["sources_sha256"]):
         traffic = PROFILED_TRAFFIC["bytes"]
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": value / PAGES_MVOX, "vs_baseline_ref": PAGES_REF, "dtype": "bf16", "data": "synthetic", "config": CONFIG,
-        "impl": "ours",
-        "layer_ms_mean": statistics.mean(layer_ms), "layer_ms_min": min(layer_ms),
-        "layer_ms_median": statistics.median(layer_ms),
-        # first layer of every step: L2 was flushed just before it
-        "layer_ms_cold_l2_median": statistics.median(layer_ms[0::LAYERS]),
+        "scaling": "weak", "vs_baseline": value / PAGES_MVOX, "vs_baseline_ref": PAGES_REF, "dtype": "bf16",
+        "data": "synthetic", "config": CONFIG, "impl": "ours",
+        # per layer: a step's time / 10 (the ten launches of one graph replay)
+        "layer_ms_median": layer_s * 1e3, "layer_ms_min": min(step_ms) / LAYERS,
         "map_build_ms": statistics.median(build_ms), "pairs": pairs,
         # build floor: coords read once + one 4-byte index per non-centre pair
         "map_build_floor_gbs": (16 * n + 4 * (pairs - n)) / (statistics.median(build_ms) / 1e3) / 1e9,
-        "tile_rows": m.tile_rows, "mma_columns_useful_frac": col_eff,
-        "roofline": {"bound": "hbm" if t_hbm >= t_tensor else "tensor", "achieved": achieved_gbs,
-                     "peak": hbm, "unit": "GB/s", "frac": achieved_gbs / hbm, "traffic": traffic,
-                     "kernel": kname, "algorithmic_bytes_per_launch": byts,
-                     "useful_flops_per_launch": flops, "t_hbm_us": t_hbm * 1e6, "t_tensor_us": t_tensor * 1e6,
-                     "frac_of_roofline_time": max(t_hbm, t_tensor) / avg_launch_s,
-                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback"},
+        "tile_rows": st["rows_per_tile"], "tiles": st["tiles"], "spans": st["spans"],
+        "issued_column_efficiency": issued_column_efficiency(pairs, st["tiles"] * st["rows_per_tile"], st["span_cols"]),
+        "roofline": {"bound": rf["bound"], "achieved": rf["achieved_gbs"] if rf["bound"] == "hbm" else rf["achieved_tflops"],
+                     "peak": hbm if rf["bound"] == "hbm" else tf_burst, "unit": "GB/s" if rf["bound"] == "hbm" else "TFLOP/s",
+                     "frac": rf["frac"], "traffic": traffic, "kernel": kname,
+                     "algorithmic_bytes_per_launch": rf["algorithmic_bytes"],
+                     "useful_flops_per_launch": rf["useful_flops"], "t_roofline_us": rf["t_roof_us"],
+                     "achieved_gbs": rf["achieved_gbs"], "achieved_tflops": rf["achieved_tflops"],
+                     "peak_source": (f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs / bf16_tflops)" if peak_kind == "measured"
+                                     else "fallback (6650 GB/s, 1590 TFLOP/s)")},
         "clocks": clocks,
+        # the timed region's kernels: one forward launch per layer, replayed from the graph
         "gpu_launches": args.steps * LAYERS,
+        # the library's per-map counters of the calls made through the API (warm-up and
+        # capture; replays bypass the library): which kernel the layers use
+        "launch_counts": counts,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_total / args.steps,
                 "includes": "H2D coords+features+weights, map build, 10 layers, D2H output"},
     }
+    if per_config is not None:
+        line["per_config"] = per_config
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(workloads.make_workload(WORKLOAD, 0, n_layers=1))
+        wl1 = workloads.make_workload(WORKLOAD, 0, n_layers=1)
+        line["cpu_baseline"] = cpu_oracle_sample(wl1, wl1.layers[0], 10.0)
     print(json.dumps(line), flush=True)
 
 
@@ -395,6 +502,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

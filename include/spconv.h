@@ -195,7 +195,9 @@ SPCONV_API spconv_status_t spconv_map_stats(spconv_map_t map, spconv_map_stats_t
 
 /*
  * Synchronise `stream` and report (then clear) any device-side wait of a forward
- * kernel on this map that gave up: SPCONV_OK or SPCONV_ERR_TIMEOUT.
+ * kernel on this map that gave up: SPCONV_OK or SPCONV_ERR_TIMEOUT.  After a
+ * timeout it also resets the map's tile-scheduler counters; call it before the
+ * map's next forward.
  */
 SPCONV_API spconv_status_t spconv_map_check(spconv_map_t map, void* stream);
 

@@ -103,8 +103,8 @@ struct MapData {
     int32_t* idx_stream = nullptr;
     int64_t* idx_off = nullptr;
     int64_t max_tile_cols = 0;
-    // work counters of the forward's tile scheduler: a launch takes slot
-    // (launch number % kSchedSlots), cleared on its stream just before it
+    // work counters of the forward's tile scheduler: launches take the slots in
+    // turn; the build zeroes them and each launch leaves its slot at zero
     uint32_t* sched = nullptr;
     int32_t* win_order = nullptr;  // [win_tiles] tiles in claim order (most expensive first)
     int64_t win_spans = 0;         // spans over all tiles (MMA jobs besides the centre)

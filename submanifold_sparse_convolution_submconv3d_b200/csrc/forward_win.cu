@@ -35,7 +35,8 @@
 //               fill for holes) into the swizzled K-major layout the MMA reads, so
 //               each unit's uses are filled and drained strictly in turn
 //   warps 6-13  epilogue: two warps per TMEM lane quarter, alternate 32-column
-//               chunks: accumulator + bias -> bf16, staged in shared memory, then
+//               chunks (warp w covers lanes 32 (w % 4) .. +31, the hardware's rule
+//               for TMEM access): accumulator + bias -> bf16, staged in shared memory, then
 //               16-byte stores to each output row, written exactly once; output
 //               rows and bias are fetched before the accumulator is ready
 // Every wait is bounded: after kWaitTimeoutNs the kernel records kFwdErrTimeout
@@ -53,8 +54,11 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kWarpMma = 0, kWarpTma = 1, kWarpGather0 = 2, kGatherWarps = 4, kWarpEpi0 = 6, kEpiWarps = 8;
+constexpr int kWarpMma = 0, kWarpTma = 1, kWarpGather0 = 2, kGatherWarps = 4, kEpiWarps = 8;
+constexpr int kWarpEpi0 = kWarpGather0 + kGatherWarps;
 constexpr int kThreads = 32 * (kWarpEpi0 + kEpiWarps);  // 448
+constexpr int kEpiGroups = kEpiWarps / 4;  // epilogue warps per TMEM lane quarter
+static_assert(kEpiWarps % 4 == 0 && kWinMaxRows / 32 % kEpiGroups == 0, "whole lane quarters, whole chunks");
 constexpr int kAccBufs = 2;
 constexpr int kIdxBufs = 2;
 constexpr int kTileSlots = 4;          // tile-record ring
@@ -87,8 +91,10 @@ struct WinLayout {
     static constexpr int kThreadsPerRow = KC * 2 / 16;         // 16-byte chunks of one row's chunk
     static constexpr int kWarpRows = 32 / kThreadsPerRow;      // rows one warp instruction covers
     static constexpr int kSliceRows = kUnitRows / kGatherWarps;  // rows of a unit one gather warp fills
-    static constexpr int kPasses = kSliceRows / kWarpRows;
-    static_assert(kPasses >= 1 && kSliceRows % kWarpRows == 0, "a slice must split into whole passes");
+    // passes of one warp instruction over a slice; when one instruction covers more
+    // rows than a slice holds, the lanes past the slice stay idle
+    static constexpr int kPasses = (kSliceRows + kWarpRows - 1) / kWarpRows;
+    static_assert(kSliceRows % kWarpRows == 0 || kWarpRows % kSliceRows == 0, "slices and passes must align");
     static constexpr int kChunksPerAtom = kARB / 16;
     static constexpr uint32_t kSwz = kARB / 16 - 1;
     static constexpr uint32_t kBLayout = kARB == 128 ? 2u : (kARB == 64 ? 4u : 6u);
@@ -119,7 +125,7 @@ struct WinParams {
     const uint32_t* recs;       // [tiles][kWinJobStride] tile records (null for kernel size 1)
     const int32_t* idx_stream;  // per-tile source rows of every job (null for kernel size 1)
     const int32_t* order;       // [tiles] claim order of the tiles (null: natural order)
-    unsigned int* work;         // this launch's work counter, zero at launch
+    unsigned int* work;         // this launch's work counter: zero at launch, left at zero
     int64_t n, tiles;
     int rows;                   // rows per tile (multiple of 16, <= 256)
     int cblocks;                // output-channel blocks of BM
@@ -361,6 +367,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const unsigned int c = atomicAdd(p.work, 1u);  // claim number: tile order, then channel block
                 int* su = reinterpret_cast<int*>(slot);
                 if ((int64_t)c >= units) {
+                    // every CTA claims until its first miss, so a launch makes exactly
+                    // units + gridDim.x claims; the CTA that makes the last one knows
+                    // that no claim is pending and sets the counter back to zero for
+                    // the next launch that uses it
+                    if ((int64_t)c == units + gridDim.x - 1) atomicExch(p.work, 0u);
                     su[0] = -1;
                     mbar_arrive(tileF0 + 8 * s);
                     return false;
@@ -517,6 +528,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                (uint32_t)(unit * L::kUnitAtomBytes);
 #pragma unroll
                         for (int pp = 0; pp < L::kPasses; ++pp) {
+                            if (L::kWarpRows > L::kSliceRows && prow >= L::kSliceRows) continue;
                             const uint32_t lin =
                                 (uint32_t)((g * L::kSliceRows + prow + pp * L::kWarpRows) * L::kARB + qa * 16);
                             cp_async_16(ubase + (lin ^ (((lin >> 7) & L::kSwz) << 4)),
@@ -539,11 +551,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ------------------------------------------------ epilogue
         const int quarter = warp & 3;
-        const int half = (warp - kWarpEpi0) >> 2;
+        const int half = (warp - kWarpEpi0) >> 2;  // this warp's group within its lane quarter
         const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
         __nv_bfloat16* stg = stage + (warp - kWarpEpi0) * L::kStageRows * L::kChPerWarp;
         constexpr int kVecPerRow = L::kChPerWarp * 2 / 16;
-        constexpr int kChunksPerWarp = kWinMaxRows / 32 / 2;  // this warp's 32-column chunks of a tile
+        constexpr int kChunksPerWarp = kWinMaxRows / 32 / kEpiGroups;  // this warp's 32-column chunks of a tile
         const bool lane_ok = lane < L::kChPerWarp;
         for (int i = 0; !aborted; ++i) {
             const int s = i % kTileSlots;
@@ -567,7 +579,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int orow[kChunksPerWarp];
 #pragma unroll
             for (int c4 = 0; c4 < kChunksPerWarp; ++c4) {
-                const int col = (half + 2 * c4) * 32 + lane;
+                const int col = (half + kEpiGroups * c4) * 32 + lane;
                 orow[c4] = col < t_eff ? (p.perm ? p.perm[row_t0 + col] : (int)(row_t0 + col)) : -1;
             }
             const float bv = (p.bias && lane_ok) ? __bfloat162float(p.bias[ch_base + lane]) : 0.0f;
@@ -578,7 +590,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
 #pragma unroll
             for (int c4 = 0; c4 < kChunksPerWarp; ++c4) {
-                const int cc = half + 2 * c4;
+                const int cc = half + kEpiGroups * c4;
                 if (cc * 32 < t_eff) {
                     float v[32];
                     tmem_ld_x32(tmem + lane_base + (uint32_t)buf * kAccCols + (uint32_t)(cc * 32), v);
@@ -715,14 +727,10 @@ spconv_status_t launch(const MapData& m, const void* x, int cin, const void* w, 
             attr_done[dev] = 1;
         }
     }
-    // this launch's work counter: one of the map's slots, cleared on the stream
+    // this launch's work counter: one of the map's slots in turn (zeroed by the
+    // build, and set back to zero by the launch's last claim)
     static std::atomic<uint64_t> launches{0};
     unsigned int* work = m.sched + (launches.fetch_add(1) % kSchedSlots);
-    cudaError_t me = cudaMemsetAsync(work, 0, sizeof(unsigned int), stream);
-    if (me != cudaSuccess) {
-        *ce = me;
-        return SPCONV_ERR_CUDA;
-    }
     WinParams p;
     p.perm = kvol == kVol3 ? m.perm : nullptr;
     p.recs = kvol == kVol3 ? m.win_jobs : nullptr;

@@ -211,6 +211,7 @@ spconv_status_t spconv_build_map(const int32_t* coords, int64_t n, const int32_t
     }
     e = al.err;
     if (e == cudaSuccess) e = cudaMemsetAsync(d.fwd_err, 0, sizeof(unsigned int), stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(d.sched, 0, spconv::kSchedSlots * sizeof(uint32_t), stream);
     if (e == cudaSuccess)
         e = spconv::launch_build_map(coords, n, extent, kernel_size, table, slots, d.nbr, keys[0], flags, stream);
     if (e == cudaSuccess && k3) {
@@ -288,6 +289,9 @@ spconv_status_t spconv_map_check(spconv_map_t map, void* stream_) {
     cudaError_t e = cudaMemcpyAsync(&err, map->d.fwd_err, sizeof(err), cudaMemcpyDeviceToHost, stream);
     if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
     if (e == cudaSuccess && err) e = cudaMemsetAsync(map->d.fwd_err, 0, sizeof(unsigned int), stream);
+    // a forward that gave up may have left its work counter mid-count
+    if (e == cudaSuccess && err && map->d.sched)
+        e = cudaMemsetAsync(map->d.sched, 0, spconv::kSchedSlots * sizeof(uint32_t), stream);
     if (e != cudaSuccess) return fail_cuda(e, "spconv_map_check");
     if (err & spconv::kFwdErrTimeout) return fail(SPCONV_ERR_TIMEOUT, "a device-side wait in a forward kernel gave up");
     return SPCONV_OK;

@@ -11,29 +11,22 @@ sys.path.insert(0, ROOT)
 import bench  # noqa: E402
 
 
-def _map(rows: int, hits_per_offset: dict) -> np.ndarray:
-    """[rows, 27] map: the centre always hits; offset k hits its first hits_per_offset[k] rows."""
-    nbr = np.full((rows, 27), -1, dtype=np.int32)
-    nbr[:, 13] = np.arange(rows)
-    for k, h in hits_per_offset.items():
-        nbr[:h, k] = 0
-    return nbr
+def test_issued_column_efficiency():
+    # 3 tiles of 16 rows (48 issued centre columns) and 32 span columns for 40 pairs
+    assert bench.issued_column_efficiency(pairs=40, npad=48, span_cols=32) == pytest.approx(40 / 80)
+    assert bench.issued_column_efficiency(pairs=0, npad=0, span_cols=0) == 1.0
 
 
-def test_column_efficiency_full_jobs_is_one():
-    # one 48-row tile, every offset full: every job is exactly 48 columns
-    nbr = _map(48, {k: 48 for k in range(27) if k != 13})
-    assert bench.mma_column_efficiency(nbr, tile_rows=48, bm=128) == 1.0
-
-
-def test_column_efficiency_counts_padding():
-    # 48-row tile: centre 48 columns (48 issued), offset 0 has 10 hits -> 16 issued,
-    # offset 5 has 40 hits -> 48 issued, others none
-    nbr = _map(48, {0: 10, 5: 40})
-    assert bench.mma_column_efficiency(nbr, tile_rows=48) == pytest.approx((48 + 10 + 40) / (48 + 16 + 48))
-    # two tiles of 24 rows: centre 24 + 24 (rounded to 32 each); offset 0: 10 in tile 0 -> 16
-    nbr = _map(48, {0: 10})
-    assert bench.mma_column_efficiency(nbr, tile_rows=24) == pytest.approx((48 + 10) / (32 + 32 + 16))
+def test_roofline_picks_the_slower_bound():
+    # 10 voxels, 30 pairs, 16 -> 32 channels: bytes vs FLOPs at chosen peaks
+    byts, flops = bench.roofline_bytes_flops(n=10, pairs=30, cin=16, cout=32)
+    r = bench.roofline(10, 30, 16, 32, 27, layer_s=1e-6, hbm_gbs=byts / 1e3, tflops=flops / 1e6 * 2)
+    assert r["bound"] == "hbm" and r["t_roof_us"] == pytest.approx(1.0) and r["frac"] == pytest.approx(1.0)
+    r = bench.roofline(10, 30, 16, 32, 27, layer_s=2e-6, hbm_gbs=byts / 1e3 * 4, tflops=flops / 1e6)
+    assert r["bound"] == "tensor" and r["frac"] == pytest.approx(0.5)
+    # kernel size 1: the weights are one [Cin, Cout] matrix and no neighbour indices
+    b1, f1 = bench.roofline_bytes_flops(n=10, pairs=10, cin=16, cout=32, kvol=1)
+    assert b1 == 10 * 16 * 2 + 16 * 32 * 2 + 32 * 2 + 10 * 32 * 2 and f1 == 2 * 16 * 32 * 10
 
 
 def test_roofline_bytes_and_flops():
@@ -99,18 +92,3 @@ def test_tc_kernel_name_follows_the_dispatch():
     assert bench.tc_kernel_name(64, 64) == "k_subm_win<64,64>"
     assert bench.tc_kernel_name(48, 192) == "k_subm_win<64,16>"
     assert bench.tc_kernel_name(32, 256) == "k_subm_win<128,32>"
-
-
-def test_column_efficiency_of_the_bench_workload():
-    """The bench reports the fraction of issued MMA columns that carry a pair. On the
-    128^3 / 10 % workload, with the 355-row tiles the library picks on 148 SMs
-    (ceil(209715 / (384 * 148)) = 4 waves, ceil(209715 / (4 * 148)) = 355 rows),
-    the oracle's map gives 85.4 %."""
-    import oracle
-    import workloads
-
-    wl = workloads.make_workload("uniform", 0, n_layers=1)
-    nbr = oracle.neighbor_map(wl.coords, wl.grid)
-    assert -(-wl.n // (384 * 148)) == 4 and -(-wl.n // (4 * 148)) == 355
-    assert int((nbr >= 0).sum()) == 745983
-    assert bench.mma_column_efficiency(nbr, 355) == pytest.approx(0.8541, abs=1e-4)

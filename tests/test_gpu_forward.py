@@ -239,14 +239,17 @@ def test_uniform_full_output_every_row(sp):
 
 
 def test_repeat_calls_identical(sp):
+    """Many launches on one map reuse its tile-scheduler counters in turn (each
+    launch leaves its counter at zero): every output must be the same."""
     coords, ext, x, w, b = _case(9, 20, 2500, 128, 128)
     m = sp.spconv_build_map(coords_dev(coords), ext, 3)
     try:
         xd, wd, bd = to_dev(x, "bf16"), to_dev(w, "bf16"), to_dev(b, "bf16")
         o1 = sp.spconv_subm_forward(m, xd, wd, bd)
-        o2 = sp.spconv_subm_forward(m, xd, wd, bd)
+        outs = [sp.spconv_subm_forward(m, xd, wd, bd) for _ in range(130)]  # > 2 x the 64 counter slots
         m.check()
-        assert torch.equal(o1, o2)
+        assert all(torch.equal(o1, o) for o in outs)
+        assert_close(o1, _ref(coords, ext, x, w, b), "bf16", label="repeat")
     finally:
         m.free()
 
