@@ -19,8 +19,13 @@
 // holds two accumulators of 256 columns (lane = output channel, column = sorted
 // row of the tile), so the epilogue of one tile overlaps the MMAs of the next.
 //
-// Warp roles (448 threads):
-//   warp 0      TMEM allocator; lane 0 issues every tcgen05.mma and commit
+// Warp roles (480 threads):
+//   warp 0      TMEM allocator; lane 0 issues every tcgen05.mma and commit, from
+//               commands the preparer posts (issuing blocks while the tensor pipe
+//               is busy, so the issuer does nothing else)
+//   warp 14     lane 0: MMA preparer: per (job, chunk) waits for the accumulator,
+//               the weight tile and the gathered units, places the job in the B
+//               ring and posts the command
 //   warp 1      lane 0: claims units (tiles in the map's claim order, most
 //               expensive first) and copies each unit's tile record (job list and
 //               index-stream position) into a ring of four shared-memory slots,
@@ -56,7 +61,13 @@ using namespace sm100;
 
 constexpr int kWarpMma = 0, kWarpTma = 1, kWarpGather0 = 2, kGatherWarps = 4, kEpiWarps = 8;
 constexpr int kWarpEpi0 = kWarpGather0 + kGatherWarps;
-constexpr int kThreads = 32 * (kWarpEpi0 + kEpiWarps);  // 448
+constexpr int kWarpPrep = kWarpEpi0 + kEpiWarps;        // 14
+constexpr int kThreads = 32 * (kWarpPrep + 1);          // 480
+// MMA command ring from the preparer to the issuer: per (job, chunk) two uint4,
+// {A descriptor, B descriptor} and {TMEM column, instruction descriptor,
+// B units | unit count << 8 | weight slot << 16 | flags << 24, accumulator buffer}.
+constexpr int kCmdSlots = 16;
+constexpr uint32_t kCmdRelA = 1, kCmdInit = 2, kCmdFirst = 4, kCmdTileEnd = 8, kCmdExit = 16;
 constexpr int kEpiGroups = kEpiWarps / 4;  // epilogue warps per TMEM lane quarter
 static_assert(kEpiWarps % 4 == 0 && kWinMaxRows / 32 % kEpiGroups == 0, "whole lane quarters, whole chunks");
 constexpr int kAccBufs = 2;
@@ -112,11 +123,11 @@ struct WinLayout {
     __host__ __device__ static int idx_buf_bytes(int max_cols) { return round_up((max_cols + kUnitRows) * 4, 128); }
     __host__ __device__ static int ring_bytes(int sa, int ub) { return sa * kAPad + ub * kUnitBytes; }
     __host__ __device__ static int num_bars(int sa, int ub) {
-        return 2 * sa + 2 * ub + 2 * kAccBufs + 2 * kIdxBufs + 2 * kTileSlots + 1;
+        return 2 * sa + 2 * ub + 2 * kAccBufs + 2 * kIdxBufs + 2 * kTileSlots + 2 * kCmdSlots + 1;
     }
     __host__ __device__ static int smem_bytes(int sa, int ub, int max_cols) {
         return 1024 + ring_bytes(sa, ub) + kStageBytes + kIdxBufs * idx_buf_bytes(max_cols) +
-               kTileSlots * kSlotBytes + num_bars(sa, ub) * 8 + 16;
+               kTileSlots * kSlotBytes + kCmdSlots * 32 + num_bars(sa, ub) * 8 + 16;
     }
 };
 
@@ -211,7 +222,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(b_ring + UB * L::kUnitBytes);
     int32_t* idx_buf = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(stage) + L::kStageBytes);
     uint8_t* tile_ring = reinterpret_cast<uint8_t*>(idx_buf + kIdxBufs * p.idx_buf_elems);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(tile_ring + kTileSlots * kSlotBytes);
+    uint4* cmd_ring = reinterpret_cast<uint4*>(tile_ring + kTileSlots * kSlotBytes);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(cmd_ring + 2 * kCmdSlots);
     int* misc = reinterpret_cast<int*>(bars + L::num_bars(SA, UB));
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
     volatile int* abort_flag = misc + 1;
@@ -221,7 +233,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t accF0 = emptyB0 + 8 * UB, accE0 = accF0 + 8 * kAccBufs;
     const uint32_t idxF0 = accE0 + 8 * kAccBufs, idxE0 = idxF0 + 8 * kIdxBufs;
     const uint32_t tileF0 = idxE0 + 8 * kIdxBufs, tileE0 = tileF0 + 8 * kTileSlots;
-    const uint32_t drain = tileE0 + 8 * kTileSlots;
+    const uint32_t cmdF0 = tileE0 + 8 * kTileSlots, cmdE0 = cmdF0 + 8 * kCmdSlots;
+    const uint32_t drain = cmdE0 + 8 * kCmdSlots;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nchunks = p.cin / KC;
@@ -248,6 +261,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(tileF0 + 8 * s, 1);
             mbar_init(tileE0 + 8 * s, kTileConsumers);
         }
+        for (int s = 0; s < kCmdSlots; ++s) {
+            mbar_init(cmdF0 + 8 * s, 1);
+            mbar_init(cmdE0 + 8 * s, 1);
+        }
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -264,11 +281,69 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == kWarpMma) {
         // ------------------------------------------------ tcgen05.mma issuer (lane 0)
+        // Issuing blocks while the tensor pipe is busy, so this thread does nothing
+        // else: it takes each (job, chunk) command the preparer posted, issues the
+        // MMAs and the commits that release the operands, and moves on.
+        if (lane == 0) {
+            for (int cq = 0;; ++cq) {
+                const int s = cq % kCmdSlots;
+                if (!wait_bar<kSleepMma>(cmdF0 + 8 * s, (uint32_t)(cq / kCmdSlots) & 1u, abort_flag, p.err)) {
+                    aborted = true;
+                    break;
+                }
+                const uint4 c0 = cmd_ring[2 * s], c1 = cmd_ring[2 * s + 1];
+                mbar_arrive(cmdE0 + 8 * s);  // the command is in registers now
+                const uint32_t fl = c1.z >> 24;
+                if (fl & kCmdExit) break;
+                if (fl & kCmdFirst) tc_fence_after();  // the epilogue's reads of this accumulator are done
+                // the B units were written by cp.async (generic proxy); the MMA reads
+                // them through the async proxy
+                fence_proxy_async_smem();
+                const uint64_t adesc0 = (uint64_t)c0.x | ((uint64_t)c0.y << 32);
+                const uint64_t bdesc0 = (uint64_t)c0.z | ((uint64_t)c0.w << 32);
+                // later K steps add their byte offset (>> 4) to the start-address field,
+                // which cannot carry out of it because shared addresses stay below 256 KB
+#pragma unroll
+                for (int kk = 0; kk < KC / 16; ++kk) {
+                    const uint32_t boff =
+                        (uint32_t)((kk / L::kStepsPerAtom) * UB * L::kUnitAtomBytes + (kk % L::kStepsPerAtom) * 32);
+                    mma_bf16(c1.x, adesc0 + (uint64_t)((kk * 2048) >> 4), bdesc0 + (uint64_t)(boff >> 4), c1.y,
+                             ((fl & kCmdInit) && kk == 0) ? 0u : 1u);
+                }
+                const int u0 = (int)(c1.z & 0xFFu), m = (int)((c1.z >> 8) & 0xFFu), as = (int)((c1.z >> 16) & 0xFFu);
+                for (int q = 0; q < m; ++q) mma_commit(emptyB0 + 8 * (u0 + q));
+                if (fl & kCmdRelA) mma_commit(emptyA0 + 8 * as);
+                if (fl & kCmdTileEnd) mma_commit(accF0 + 8 * c1.w);
+            }
+            if (aborted) {
+                mma_commit(drain);  // wait for the MMAs in flight before TMEM is freed
+                const uint64_t t0 = globaltimer_ns();
+                while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == kWarpPrep) {
+        // ------------------------------------------------ MMA preparer (lane 0)
+        // Walks the tiles and their jobs: waits for the accumulator, the weight tile
+        // and the gathered units of each (job, chunk), places it in the B ring and
+        // posts one command per (job, chunk) to the issuer, up to kCmdSlots ahead.
         if (lane == 0) {
             int as = SA - 1;
             uint32_t aph = 1u;
             int ucur = 0;
             uint32_t bph = 0;  // bit u: phase of unit u's next use
+            int cq = 0;
+            auto post = [&](const uint4& c0, const uint4& c1) -> bool {
+                const int s = cq % kCmdSlots;
+                if (!wait_bar<kSleepMma>(cmdE0 + 8 * s, ((uint32_t)(cq / kCmdSlots) & 1u) ^ 1u, abort_flag, p.err))
+                    return false;
+                cmd_ring[2 * s] = c0;
+                cmd_ring[2 * s + 1] = c1;
+                mbar_arrive(cmdF0 + 8 * s);
+                ++cq;
+                return true;
+            };
             for (int i = 0; !aborted; ++i) {
                 const int s = i % kTileSlots;
                 const uint8_t* slot = tile_ring + s * kSlotBytes;
@@ -276,14 +351,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     aborted = true;
                     break;
                 }
-                if (slot_unit(slot) < 0) break;
+                if (slot_unit(slot) < 0) {
+                    if (!post(make_uint4(0, 0, 0, 0), make_uint4(0, 0, kCmdExit << 24, 0))) aborted = true;
+                    break;
+                }
                 const uint32_t* rec = slot_rec(slot);
                 const int buf = i & 1;
                 if (!wait_bar<kSleepMma>(accE0 + 8 * buf, ((uint32_t)(i >> 1) & 1u) ^ 1u, abort_flag, p.err)) {
                     aborted = true;
                     break;
                 }
-                tc_fence_after();
                 const uint32_t dbase = tmem + (uint32_t)buf * kAccCols;
                 const int nj = (int)rec[0];
                 int prev_k = -1;
@@ -317,39 +394,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                         }
                         if (aborted) break;
-                        // the B units were written by cp.async (generic proxy); the MMA
-                        // reads them through the async proxy
-                        fence_proxy_async_smem();
-                        // descriptors of K step 0; later steps add their byte offset (>> 4)
-                        // to the start-address field, which cannot carry out of it because
-                        // shared addresses stay below 256 KB
                         const uint64_t adesc0 = smem_desc(smem_addr(a_ring + as * L::kAPad), KC * 128, 1024, 2);
                         const uint64_t bdesc0 = smem_desc(smem_addr(b_ring) + (uint32_t)(u0 * L::kUnitAtomBytes), 16,
                                                           L::kBSbo, L::kBLayout);
-#pragma unroll
-                        for (int kk = 0; kk < KC / 16; ++kk) {
-                            const uint32_t boff = (uint32_t)((kk / L::kStepsPerAtom) * UB * L::kUnitAtomBytes +
-                                                             (kk % L::kStepsPerAtom) * 32);
-                            mma_bf16(d, adesc0 + (uint64_t)((kk * 2048) >> 4), bdesc0 + (uint64_t)(boff >> 4), idesc,
-                                     (j == 0 && c == 0 && kk == 0) ? 0u : 1u);
+                        uint32_t fl = 0;
+                        if (nchunks > 1 || last_of_k) fl |= kCmdRelA;
+                        if (j == 0 && c == 0) fl |= kCmdInit | kCmdFirst;
+                        if (j == nj - 1 && c == nchunks - 1) fl |= kCmdTileEnd;
+                        const uint4 c0 = make_uint4((uint32_t)adesc0, (uint32_t)(adesc0 >> 32), (uint32_t)bdesc0,
+                                                    (uint32_t)(bdesc0 >> 32));
+                        const uint4 c1 = make_uint4(d, idesc, (uint32_t)u0 | ((uint32_t)m << 8) |
+                                                                   ((uint32_t)as << 16) | (fl << 24),
+                                                    (uint32_t)buf);
+                        if (!post(c0, c1)) {
+                            aborted = true;
+                            break;
                         }
-                        for (int q = 0; q < m; ++q) {
-                            mma_commit(emptyB0 + 8 * (u0 + q));
-                            bph ^= 1u << (u0 + q);
-                        }
-                        if (nchunks > 1 || last_of_k) mma_commit(emptyA0 + 8 * as);
+                        for (int q = 0; q < m; ++q) bph ^= 1u << (u0 + q);
                     }
                     jw = jn;
                 }
                 if (aborted) break;
-                mma_commit(accF0 + 8 * buf);
                 mbar_arrive(tileE0 + 8 * s);
-            }
-            if (aborted) {
-                mma_commit(drain);  // wait for the MMAs in flight before TMEM is freed
-                const uint64_t t0 = globaltimer_ns();
-                while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
-                }
             }
         }
         __syncwarp();
@@ -548,7 +614,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (issuer && aborted && lane == 0) __nanosleep(200000);  // the index copy in flight lands first
         cp_async_wait_all();
-    } else {
+    } else if (warp < kWarpEpi0 + kEpiWarps) {
         // ------------------------------------------------ epilogue
         const int quarter = warp & 3;
         const int half = (warp - kWarpEpi0) >> 2;  // this warp's group within its lane quarter
