@@ -18,7 +18,21 @@ pixal3d_mrp_mlx README, "Status", for the [K^3, in, out] weight layout):
 
 with the offset order k(d) = (dx+1)*9 + (dy+1)*3 + (dz+1) (a reading: the
 pages do not fix it), cross-correlation orientation (gather p + d), batch
-isolation, and grid-boundary neighbours treated as holes.
+isolation, and grid-boundary neighbours treated as holes.  With ``flip=True``
+the map gathers p - d instead: the alternative orientation the lato.2_mrp_mlx
+README ("Correctness") leaves open and builds behind its --flip-kernel switch.
+
+The resampling ops around the convolution (``downsample``, ``downsample_amax``,
+``upsample``, ``subdivide``) follow the lato.2_mrp_mlx README ("Status":
+SparseDownsample is max pooling with the "amax" reduction; the table of upstream
+equivalents: SparseSubdivide expands the coordinates x8) and the pixal3d_mrp_mlx
+README ("Scope, measured against the shared core": SparseUpsample(2) is the
+inverse of a downsample that reuses its pairing).  Readings where the pages are
+silent: a voxel p falls in the coarse voxel floor(p / factor) of the same batch;
+the coarse voxels are listed in increasing lexicographic (b, x, y, z) order; the
+coarse grid is ceil(extent / factor); "amax" of a block is the largest value,
+with +0 above -0 (the IEEE 754 total order); subdivision lists the children of
+voxel i as rows 8 i + c, c = 4 ox + 2 oy + oz, each carrying voxel i's features.
 
 Pins: every function here is pinned by ``tests/test_oracle_pins.py`` against
 dense brute force, torch's CPU conv3d, closed forms and invariants; none is
@@ -64,6 +78,9 @@ def _load():
         lib.oracle_neighbor_map.restype = ctypes.c_int
         lib.oracle_neighbor_map.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
                                             ctypes.c_int32, ctypes.c_void_p]
+        lib.oracle_neighbor_map_oriented.restype = ctypes.c_int
+        lib.oracle_neighbor_map_oriented.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                                     ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p]
         lib.oracle_forward_f64.restype = ctypes.c_int
         lib.oracle_forward_f64.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32,
                                            ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
@@ -77,13 +94,15 @@ def _ptr(a: np.ndarray | None) -> int | None:
     return None if a is None else a.ctypes.data
 
 
-def neighbor_map(coords: np.ndarray, extent, kernel_size: int = 3) -> np.ndarray:
-    """int32 [N, K^3]: row index of the active voxel at p_i + d_k, or -1."""
+def neighbor_map(coords: np.ndarray, extent, kernel_size: int = 3, flip: bool = False) -> np.ndarray:
+    """int32 [N, K^3]: row index of the active voxel at p_i + d_k (p_i - d_k with
+    ``flip``), or -1."""
     coords = np.ascontiguousarray(coords, dtype=np.int32).reshape(-1, 4)
     ext = np.ascontiguousarray(extent, dtype=np.int32).reshape(3)
     kvol = kernel_size ** 3
     nbr = np.empty((coords.shape[0], kvol), dtype=np.int32)
-    rc = _load().oracle_neighbor_map(_ptr(coords), coords.shape[0], _ptr(ext), kernel_size, _ptr(nbr))
+    rc = _load().oracle_neighbor_map_oriented(_ptr(coords), coords.shape[0], _ptr(ext), kernel_size,
+                                              1 if flip else 0, _ptr(nbr))
     if rc != OK:
         raise OracleError(rc)
     return nbr
@@ -124,7 +143,7 @@ def _offsets(kernel_size: int):
     return [(dx, dy, dz) for dx in range(-r, r + 1) for dy in range(-r, r + 1) for dz in range(-r, r + 1)]
 
 
-def neighbor_map_py(coords, extent, kernel_size: int = 3) -> np.ndarray:
+def neighbor_map_py(coords, extent, kernel_size: int = 3, flip: bool = False) -> np.ndarray:
     coords = np.asarray(coords).reshape(-1, 4).tolist()
     ex, ey, ez = (int(v) for v in extent)
     table = {}
@@ -135,10 +154,11 @@ def neighbor_map_py(coords, extent, kernel_size: int = 3) -> np.ndarray:
             raise OracleError(DUPLICATE)
         table[(b, x, y, z)] = i
     offs = _offsets(kernel_size)
+    s = -1 if flip else 1
     nbr = np.full((len(coords), len(offs)), -1, dtype=np.int32)
     for i, (b, x, y, z) in enumerate(coords):
         for k, (dx, dy, dz) in enumerate(offs):
-            nbr[i, k] = table.get((b, x + dx, y + dy, z + dz), -1)
+            nbr[i, k] = table.get((b, x + s * dx, y + s * dy, z + s * dz), -1)
     return nbr
 
 
@@ -160,3 +180,81 @@ def forward_py(nbr, x, w, bias=None) -> np.ndarray:
                     acc[co] += xv * float(w[k, ci, co])
         out[i] = acc
     return out
+
+
+# ---------------------------------------------------------------------------
+# Resampling around the convolution: SparseDownsample (amax), SparseUpsample
+# (paired with a downsample), SparseSubdivide.
+# ---------------------------------------------------------------------------
+
+def _check_coords(coords: np.ndarray, extent) -> None:
+    ext = np.asarray(extent, dtype=np.int64).reshape(3)
+    c = coords.astype(np.int64)
+    if c.size and ((c[:, 0] < 0).any() or (c[:, 0] > 65535).any() or (c[:, 1:] < 0).any()
+                   or (c[:, 1:] >= ext).any()):
+        raise OracleError(COORD_RANGE)
+
+
+def downsample(coords, extent, factor: int = 2):
+    """Coarse voxel set of SparseDownsample(factor): returns (coarse int32 [M, 4]
+    in increasing lexicographic (b, x, y, z) order, parent int32 [N] = coarse row
+    of each input row, coarse extent ceil(extent / factor))."""
+    coords = np.asarray(coords, dtype=np.int32).reshape(-1, 4)
+    _check_coords(coords, extent)
+    cells = coords.astype(np.int64).copy()
+    cells[:, 1:] //= int(factor)
+    # np.unique over rows sorts them lexicographically: one library sort as a step
+    coarse, parent = np.unique(cells, axis=0, return_inverse=True)
+    coarse_extent = tuple(-(-int(e) // int(factor)) for e in extent)
+    return coarse.astype(np.int32).reshape(-1, 4), parent.astype(np.int32).reshape(-1), coarse_extent
+
+
+def downsample_amax(parent, n_coarse: int, x) -> np.ndarray:
+    """out[g] = element-wise max of x[i] over the rows i with parent[i] = g, where
+    +0 counts as larger than -0.  Returns x's dtype (the max is one of the inputs)."""
+    parent = np.asarray(parent, dtype=np.int64).reshape(-1)
+    x = np.asarray(x)
+    xf = x.astype(np.float64)
+    out = np.full((int(n_coarse), x.shape[1]), -np.inf)
+    np.maximum.at(out, parent, xf)
+    # signed zero: a zero maximum is +0 when any element of its block is +0
+    pos_zero = np.zeros(out.shape, dtype=bool)
+    np.logical_or.at(pos_zero, parent, (xf == 0) & ~np.signbit(xf))
+    zero = out == 0
+    out[zero & pos_zero] = 0.0
+    out[zero & ~pos_zero] = -0.0
+    return out
+
+
+def upsample(parent, x_coarse) -> np.ndarray:
+    """SparseUpsample paired with a downsample: row i gets x_coarse[parent[i]]."""
+    return np.asarray(x_coarse)[np.asarray(parent, dtype=np.int64)]
+
+
+def subdivide(coords, extent, x=None):
+    """SparseSubdivide: row 8 i + c (c = 4 ox + 2 oy + oz) is (b, 2x + ox, 2y + oy,
+    2z + oz) with voxel i's features.  Returns (coords [8N, 4], features or None)."""
+    coords = np.asarray(coords, dtype=np.int32).reshape(-1, 4)
+    _check_coords(coords, extent)
+    out = np.empty((8 * coords.shape[0], 4), dtype=np.int32)
+    for c in range(8):
+        ox, oy, oz = c >> 2, (c >> 1) & 1, c & 1
+        out[c::8, 0] = coords[:, 0]
+        out[c::8, 1] = 2 * coords[:, 1] + ox
+        out[c::8, 2] = 2 * coords[:, 2] + oy
+        out[c::8, 3] = 2 * coords[:, 3] + oz
+    xo = None if x is None else np.repeat(np.asarray(x), 8, axis=0)
+    return out, xo
+
+
+def downsample_py(coords, factor: int = 2):
+    """Pure-Python twin of ``downsample`` (dict of blocks, sorted keys), tiny inputs."""
+    blocks = {}
+    for i, (b, x, y, z) in enumerate(np.asarray(coords).reshape(-1, 4).tolist()):
+        blocks.setdefault((b, x // factor, y // factor, z // factor), []).append(i)
+    keys = sorted(blocks)
+    parent = [0] * sum(len(v) for v in blocks.values())
+    for g, key in enumerate(keys):
+        for i in blocks[key]:
+            parent[i] = g
+    return np.array(keys, dtype=np.int32).reshape(-1, 4), np.array(parent, dtype=np.int32)

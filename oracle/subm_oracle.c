@@ -22,6 +22,11 @@
  *     a map of active voxel coordinates is built first, then probed per
  *     kernel offset.
  *
+ * Orientation option: the same README section says the upstream orientation
+ * is unverified and that its --flip-kernel switch builds the alternative, which
+ * gathers feats[c-d]; oracle_neighbor_map_oriented with flip = 1 computes that
+ * map (neighbour at p_i - d_k).
+ *
  * Readings where the pages are silent:
  *   - offset order: k = (dx+1)*9 + (dy+1)*3 + (dz+1), dx slowest, matching
  *     coordinate columns (x, y, z); the centre is k = 13.  For k=1, one offset.
@@ -61,11 +66,12 @@ static int cmp_entry(const void* a, const void* b) {
     return (ka > kb) - (ka < kb);
 }
 
-/* Neighbour map: nbr[i * K^3 + k] = row of the active voxel at p_i + d_k, else -1.
+/* Neighbour map: nbr[i * K^3 + k] = row of the active voxel at p_i + s d_k, else
+ * -1, with s = +1 (flip = 0) or s = -1 (flip = 1).
  * coords is int32 [n, 4] = (b, x, y, z); extent = (X, Y, Z), each in [1, 65535].
  * Returns ORACLE_OK or an error code; on error nbr is left unspecified. */
-int oracle_neighbor_map(const int32_t* coords, int64_t n, const int32_t* extent,
-                        int32_t kernel_size, int32_t* nbr) {
+int oracle_neighbor_map_oriented(const int32_t* coords, int64_t n, const int32_t* extent,
+                                 int32_t kernel_size, int32_t flip, int32_t* nbr) {
     if (n < 0 || (n > 0 && (!coords || !nbr)) || !extent) return ORACLE_INVALID_ARG;
     if (kernel_size != 1 && kernel_size != 3) return ORACLE_INVALID_ARG;
     for (int a = 0; a < 3; ++a)
@@ -96,13 +102,14 @@ int oracle_neighbor_map(const int32_t* coords, int64_t n, const int32_t* extent,
 
     const int kvol = kernel_size * kernel_size * kernel_size;
     const int r = kernel_size / 2;
+    const int s = flip ? -1 : 1;
     for (int64_t i = 0; i < n; ++i) {
         const int32_t* c = coords + 4 * i;
         int k = 0;
         for (int dx = -r; dx <= r; ++dx)
             for (int dy = -r; dy <= r; ++dy)
                 for (int dz = -r; dz <= r; ++dz, ++k) {
-                    int64_t x = (int64_t)c[1] + dx, y = (int64_t)c[2] + dy, z = (int64_t)c[3] + dz;
+                    int64_t x = (int64_t)c[1] + s * dx, y = (int64_t)c[2] + s * dy, z = (int64_t)c[3] + s * dz;
                     int32_t found = -1;
                     if (x >= 0 && x < extent[0] && y >= 0 && y < extent[1] && z >= 0 && z < extent[2]) {
                         entry_t probe;
@@ -117,6 +124,11 @@ int oracle_neighbor_map(const int32_t* coords, int64_t n, const int32_t* extent,
     }
     free(dict);
     return ORACLE_OK;
+}
+
+int oracle_neighbor_map(const int32_t* coords, int64_t n, const int32_t* extent,
+                        int32_t kernel_size, int32_t* nbr) {
+    return oracle_neighbor_map_oriented(coords, n, extent, kernel_size, 0, nbr);
 }
 
 /* Forward pass in fp64 for the output rows listed in `rows` (all rows when rows
