@@ -79,10 +79,12 @@ typedef enum { SPCONV_F32 = 0, SPCONV_BF16 = 1 } spconv_dtype_t;
  *   stream       stream on which the build runs.
  *   out_map      receives the handle on success; untouched on failure.
  *
- * Device work: pack (b, x, y, z) into a 64-bit key and validate it; insert the
- * keys into an open-addressing hash table (linear probing, 64-bit CAS, load
- * factor <= 1/2); probe the 26 neighbours of every voxel and write the dense map
- * nbr[i*27 + k] = row of p_i + d_k, or -1.  For kernel size 3 it then prepares
+ * Device work: pack (b, x, y, z) into a 64-bit key and validate it; build a
+ * dictionary of the keys -- below 2^20 voxels an open-addressing hash table
+ * (linear probing, 64-bit CAS, load factor <= 1/2), from 2^20 voxels on the keys
+ * radix-sorted with their rows (see spconv_build_map_ex); probe the 26
+ * neighbours of every voxel and write the dense map nbr[i*27 + k] = row of
+ * p_i + d_k, or -1.  For kernel size 3 it then prepares
  * the tensor-core forward's metadata: the rows sorted (stably, on the GPU) by the
  * Gray-code rank of their 26-bit neighbour mask, the neighbour table in that
  * order, and per tile of sorted rows the MMA jobs (see spconv_map_stats).
@@ -98,6 +100,47 @@ typedef enum { SPCONV_F32 = 0, SPCONV_BF16 = 1 } spconv_dtype_t;
  */
 SPCONV_API spconv_status_t spconv_build_map(const int32_t* coords, int64_t n, const int32_t* extent,
                                  int32_t kernel_size, void* stream, spconv_map_t* out_map);
+
+/*
+ * Options of spconv_build_map_ex (bits of `flags`).
+ *
+ *   SPCONV_MAP_FLIP_KERNEL  gather x at p - d_k instead of p + d_k: the kernel
+ *                           is mirrored (a true convolution rather than a
+ *                           cross-correlation).  The lato.2_mrp_mlx README
+ *                           ("Correctness") leaves open which of the two the
+ *                           upstream library computes and builds the mirrored
+ *                           one behind its --flip-kernel switch.  The map is the
+ *                           default map with offsets k and 26 - k exchanged.
+ *   SPCONV_MAP_SORTED_KEYS  build the coordinate dictionary by radix-sorting the
+ *                           packed keys and find every neighbour by binary search,
+ *                           the "sorted-key indice map" the lato.2_mrp_mlx README
+ *                           (table of upstream equivalents) names for its port,
+ *                           instead of the hash table.  Same map, bit for bit.
+ *                           Needs 16 + sum over axes of ceil(log2(extent)) <= 62
+ *                           (SPCONV_ERR_UNSUPPORTED otherwise); never reports
+ *                           SPCONV_ERR_TABLE_FULL.
+ *   SPCONV_MAP_HASH_TABLE   build with the hash table whatever the size.
+ * With neither dictionary flag the library picks one: the hash table below
+ * 2^20 voxels, the sorted keys from 2^20 voxels on when the key bits fit (and
+ * the hash table whenever spconv_debug_set_table_slots forces a table size).
+ * Both flags together: SPCONV_ERR_INVALID_ARG.
+ */
+typedef enum {
+    SPCONV_MAP_DEFAULT = 0,
+    SPCONV_MAP_FLIP_KERNEL = 1,
+    SPCONV_MAP_SORTED_KEYS = 2,
+    SPCONV_MAP_HASH_TABLE = 4
+} spconv_map_flags_t;
+
+/*
+ * spconv_build_map with options: `flags` is a bitwise OR of spconv_map_flags_t
+ * values (an unknown bit: SPCONV_ERR_INVALID_ARG).  Everything else, including
+ * memory, synchronisation and errors, is as spconv_build_map, which is this call
+ * with flags = SPCONV_MAP_DEFAULT.  The forward runs unchanged on either map.
+ */
+SPCONV_API spconv_status_t spconv_build_map_ex(const int32_t* coords, int64_t n, const int32_t* extent,
+                                               int32_t kernel_size, uint32_t flags, void* stream,
+                                               spconv_map_t* out_map);
 
 /*
  * Run one SubMConv3d layer over a map.
@@ -294,6 +337,108 @@ SPCONV_API spconv_status_t spconv_debug_set_ring_depths(int32_t a_slots, int32_t
  */
 SPCONV_API spconv_status_t spconv_build_neighbor_map_noalloc(const int32_t* coords, int64_t n, const int32_t* extent,
                                                              int32_t* nbr_out, int64_t* pairs_out, void* stream);
+
+/*
+ * ---------------------------------------------------------------- resampling
+ * The sparse ops that change the coordinate set around the convolution: the
+ * lato.2_mrp_mlx README ("Status") lists SparseDownsample as max pooling with
+ * the "amax" reduction; its table of upstream equivalents does upsampling with
+ * SparseSubdivide, a x8 expansion of the coordinates; the pixal3d_mrp_mlx README
+ * ("Scope, measured against the shared core") has SparseUpsample(2) as the
+ * inverse of a downsample that reuses the downsample's pairing.  A convolution
+ * on the new set needs a new neighbour map (spconv_build_map).
+ */
+typedef struct spconv_downsample_s* spconv_downsample_t; /* opaque, owned by the library */
+
+/*
+ * SparseDownsample(factor) coordinates.  Every voxel (b, x, y, z) falls in the
+ * coarse voxel (b, x / factor, y / factor, z / factor) (integer division); the
+ * coarse set is the set of those, in increasing lexicographic (b, x, y, z) order,
+ * on the grid ceil(extent / factor).
+ *
+ *   coords   device int32 [n, 4] (b, x, y, z), 16-byte aligned; no duplicates
+ *            needed for correctness (a repeated voxel just joins its block twice).
+ *   n        0 <= n < 2^31.
+ *   extent   host int32 [3], each in [1, 65535].
+ *   factor   block edge, in [1, 65535] (the pages use 2).
+ *   stream   stream on which the build runs; the call synchronises it once, at
+ *            the end, to read the coarse count and the error flag.
+ *   out      receives the handle on success; untouched on failure.
+ *
+ * Device work: pack each voxel's coarse key (bit fields sized by the coarse
+ * extent), radix-sort (key, row) stably, number the runs of equal keys by a scan,
+ * write the coarse coordinates, each run's start and each fine row's parent.
+ * Memory comes from the library's stream-ordered pool, as for spconv_build_map;
+ * spconv_downsample_free returns it.
+ * Errors: SPCONV_ERR_INVALID_ARG, SPCONV_ERR_COORD_RANGE, SPCONV_ERR_OOM,
+ * SPCONV_ERR_CUDA.
+ */
+SPCONV_API spconv_status_t spconv_downsample_build(const int32_t* coords, int64_t n, const int32_t* extent,
+                                                   int32_t factor, void* stream, spconv_downsample_t* out);
+
+/*
+ * Introspection of a downsample (any pointer may be NULL):
+ *   n_fine             input voxel count n
+ *   n_coarse           coarse voxel count
+ *   coarse_extent      host int32 [3]: ceil(extent / factor)
+ *   coarse_coords_dev  device int32 [n_coarse, 4] (b, x, y, z), sorted, 16-byte
+ *                      aligned: a valid `coords` argument for spconv_build_map
+ *   parent_dev         device int32 [n]: coarse row of every input row
+ * The library owns the buffers (NULL when n = 0).
+ */
+SPCONV_API spconv_status_t spconv_downsample_info(spconv_downsample_t ds, int64_t* n_fine, int64_t* n_coarse,
+                                                  int32_t* coarse_extent, const int32_t** coarse_coords_dev,
+                                                  const int32_t** parent_dev);
+
+/*
+ * Max pooling over a downsample: out[g, c] = max over input rows i with
+ * parent[i] = g of x[i, c] ("amax").  Exact; where the maximum is a zero, +0
+ * wins over -0 (the IEEE 754 total order).  NaN inputs give unspecified values.
+ *
+ *   x        device [n, channels] of dtype, row-major, 16-byte aligned.
+ *   out      device [n_coarse, channels] of dtype, 16-byte aligned; must not
+ *            overlap x.
+ * Asynchronous on `stream` (no synchronisation).  The current device must be the
+ * handle's.  Errors: SPCONV_ERR_INVALID_ARG, SPCONV_ERR_CUDA.
+ */
+SPCONV_API spconv_status_t spconv_downsample_amax(spconv_downsample_t ds, spconv_dtype_t dtype, const void* x,
+                                                  int32_t channels, void* out, void* stream);
+
+/*
+ * SparseUpsample paired with a downsample: out[i, :] = x_coarse[parent[i], :],
+ * back on the downsample's input voxels, in their input order.
+ *
+ *   x_coarse  device [n_coarse, channels] of dtype, 16-byte aligned.
+ *   out       device [n, channels] of dtype, 16-byte aligned.
+ * Asynchronous; same errors as spconv_downsample_amax.
+ */
+SPCONV_API spconv_status_t spconv_upsample(spconv_downsample_t ds, spconv_dtype_t dtype, const void* x_coarse,
+                                           int32_t channels, void* out, void* stream);
+
+/* Release a downsample (synchronises its device first, like spconv_free).  NULL
+ * is accepted and ignored. */
+SPCONV_API spconv_status_t spconv_downsample_free(spconv_downsample_t ds);
+
+/*
+ * SparseSubdivide: every voxel becomes its 8 children on the grid 2 * extent.
+ * Output row 8 i + c, c = 4 ox + 2 oy + oz with ox, oy, oz in {0, 1}, is the
+ * voxel (b, 2x + ox, 2y + oy, 2z + oz) and carries row i's features.
+ *
+ *   coords      device int32 [n, 4] (b, x, y, z), 16-byte aligned.
+ *   n           0 <= n <= 2^28.
+ *   extent      host int32 [3], each in [1, 32767] (the doubled grid must stay
+ *               within 65535).
+ *   dtype, x, channels   device features [n, channels], or x = NULL and
+ *               x_out = NULL to expand the coordinates only.
+ *   coords_out  device int32 [8n, 4], 16-byte aligned.
+ *   x_out       device [8n, channels] of dtype, 16-byte aligned.
+ *   stream      the call synchronises it once, to read the range check.
+ * Errors: SPCONV_ERR_INVALID_ARG, SPCONV_ERR_COORD_RANGE (a coordinate outside
+ * [0, extent); the outputs are then unspecified), SPCONV_ERR_OOM, SPCONV_ERR_CUDA.
+ */
+SPCONV_API spconv_status_t spconv_subdivide(const int32_t* coords, int64_t n, const int32_t* extent,
+                                            spconv_dtype_t dtype, const void* x, int32_t channels,
+                                            int32_t* coords_out, void* x_out, void* stream);
 
 #ifdef __cplusplus
 }

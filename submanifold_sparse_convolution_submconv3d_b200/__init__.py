@@ -7,9 +7,13 @@ library has not been built (``python -m submanifold_sparse_convolution_submconv3
 
 The functions carry the C names:
 
-* ``spconv_build_map(coords, extent, kernel_size=3)`` -> ``SubmMap``
+* ``spconv_build_map(coords, extent, kernel_size=3, flip_kernel=False, sorted_keys=False)``
+  -> ``SubmMap`` (``spconv_build_map_ex`` when an option is set)
 * ``spconv_subm_forward(map, x, w, bias=None, out=None)`` -> ``out``
 * ``spconv_free(map)``
+* ``spconv_downsample_build(coords, extent, factor=2)`` -> ``Downsample``;
+  ``spconv_downsample_amax(ds, x)``, ``spconv_upsample(ds, x_coarse)``
+* ``spconv_subdivide(coords, extent, x=None)`` -> ``(coords_out, x_out)``
 """
 from __future__ import annotations
 
@@ -22,6 +26,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libspconv_b200.so")
 
 OK, INVALID_ARG, UNSUPPORTED, COORD_RANGE, DUPLICATE, TABLE_FULL, OOM, CUDA_ERROR, TIMEOUT = range(9)
+MAP_DEFAULT, MAP_FLIP_KERNEL, MAP_SORTED_KEYS, MAP_HASH_TABLE = 0, 1, 2, 4
 ALGO_AUTO, ALGO_SIMT, ALGO_TCGEN05 = 0, 1, 2
 KERNEL_SIMT, KERNEL_TCGEN05 = 0, 1
 KERNEL_NAMES = ("simt", "tcgen05")
@@ -31,7 +36,9 @@ EXPORTED = ("spconv_build_map", "spconv_subm_forward", "spconv_free", "spconv_ma
             "spconv_map_tile_rows",
             "spconv_last_error", "spconv_subm_forward_algo", "spconv_debug_set_table_slots",
             "spconv_debug_set_tile_rows", "spconv_build_neighbor_map_noalloc", "spconv_map_launch_counts",
-            "spconv_map_stats", "spconv_debug_set_ring_depths")
+            "spconv_map_stats", "spconv_debug_set_ring_depths", "spconv_build_map_ex", "spconv_downsample_build",
+            "spconv_downsample_info", "spconv_downsample_amax", "spconv_upsample", "spconv_downsample_free",
+            "spconv_subdivide")
 
 
 class _MapStats(ctypes.Structure):
@@ -66,11 +73,21 @@ def _load() -> ctypes.CDLL:
     lib.spconv_map_launch_counts.argtypes = [vp, ctypes.POINTER(i64), i32]
     lib.spconv_map_stats.argtypes = [vp, ctypes.POINTER(_MapStats)]
     lib.spconv_debug_set_ring_depths.argtypes = [i32, i32]
+    lib.spconv_build_map_ex.argtypes = [vp, i64, vp, i32, ctypes.c_uint32, vp, ctypes.POINTER(vp)]
+    lib.spconv_downsample_build.argtypes = [vp, i64, vp, i32, vp, ctypes.POINTER(vp)]
+    lib.spconv_downsample_info.argtypes = [vp, ctypes.POINTER(i64), ctypes.POINTER(i64), vp, ctypes.POINTER(vp),
+                                           ctypes.POINTER(vp)]
+    lib.spconv_downsample_amax.argtypes = [vp, ctypes.c_int, vp, i32, vp, vp]
+    lib.spconv_upsample.argtypes = [vp, ctypes.c_int, vp, i32, vp, vp]
+    lib.spconv_downsample_free.argtypes = [vp]
+    lib.spconv_subdivide.argtypes = [vp, i64, vp, ctypes.c_int, vp, i32, vp, vp, vp]
     lib.spconv_last_error.restype = ctypes.c_char_p
     for name in ("spconv_build_map", "spconv_subm_forward", "spconv_subm_forward_algo", "spconv_free",
                  "spconv_map_info", "spconv_map_check", "spconv_map_tile_rows", "spconv_debug_set_table_slots",
                  "spconv_debug_set_tile_rows", "spconv_build_neighbor_map_noalloc", "spconv_map_launch_counts",
-                 "spconv_map_stats", "spconv_debug_set_ring_depths"):
+                 "spconv_map_stats", "spconv_debug_set_ring_depths", "spconv_build_map_ex",
+                 "spconv_downsample_build", "spconv_downsample_info", "spconv_downsample_amax", "spconv_upsample",
+                 "spconv_downsample_free", "spconv_subdivide"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -171,17 +188,31 @@ class SubmMap:
             pass
 
 
-def spconv_build_map(coords: torch.Tensor, extent, kernel_size: int = 3, stream=None) -> SubmMap:
-    """Build the neighbour map of int32 [N, 4] (b, x, y, z) CUDA coordinates."""
-    _require()
+def _coords_arg(coords: torch.Tensor) -> torch.Tensor:
     if coords.dtype != torch.int32 or not coords.is_cuda or coords.dim() != 2 or coords.shape[1] != 4:
         raise ValueError("coords must be a CUDA int32 tensor of shape [N, 4]")
-    coords = coords.contiguous()
+    return coords.contiguous()
+
+
+def spconv_build_map(coords: torch.Tensor, extent, kernel_size: int = 3, stream=None, flip_kernel: bool = False,
+                     sorted_keys: bool | None = None) -> SubmMap:
+    """Build the neighbour map of int32 [N, 4] (b, x, y, z) CUDA coordinates.
+    ``flip_kernel`` gathers p - d_k; ``sorted_keys`` True / False forces the sorted-key
+    or the hash-table dictionary (same map); None lets the library choose by size."""
+    _require()
+    coords = _coords_arg(coords)
     ext = (ctypes.c_int32 * 3)(*[int(v) for v in extent])
     handle = ctypes.c_void_p()
+    flags = (MAP_FLIP_KERNEL if flip_kernel else 0) | \
+        {None: 0, True: MAP_SORTED_KEYS, False: MAP_HASH_TABLE}[sorted_keys]
     with torch.cuda.device(coords.device):
-        _check(lib.spconv_build_map(coords.data_ptr() if coords.numel() else None, coords.shape[0], ext,
-                                    kernel_size, _stream(stream), ctypes.byref(handle)))
+        ptr = coords.data_ptr() if coords.numel() else None
+        if flags:
+            _check(lib.spconv_build_map_ex(ptr, coords.shape[0], ext, kernel_size, flags, _stream(stream),
+                                           ctypes.byref(handle)))
+        else:
+            _check(lib.spconv_build_map(ptr, coords.shape[0], ext, kernel_size, _stream(stream),
+                                        ctypes.byref(handle)))
     return SubmMap(handle.value, coords.device)
 
 
@@ -248,6 +279,122 @@ def spconv_build_neighbor_map_noalloc(coords: torch.Tensor, extent, out: torch.T
     return out, pairs.value
 
 
+class Downsample:
+    """Owns a downsample handle (spconv_downsample_build): the coarse voxel set and
+    the pairing of input voxels with coarse voxels."""
+
+    def __init__(self, handle: int, device: torch.device):
+        self.handle = handle
+        self.device = device
+        nf, nc, ext = ctypes.c_int64(), ctypes.c_int64(), (ctypes.c_int32 * 3)()
+        cptr, pptr = ctypes.c_void_p(), ctypes.c_void_p()
+        _check(lib.spconv_downsample_info(handle, ctypes.byref(nf), ctypes.byref(nc), ext, ctypes.byref(cptr),
+                                          ctypes.byref(pptr)))
+        self.n, self.n_coarse, self.coarse_extent = nf.value, nc.value, tuple(ext)
+        self._coarse_ptr, self._parent_ptr = cptr.value, pptr.value
+
+    def _copy(self, ptr, shape) -> torch.Tensor:
+        out = torch.empty(shape, dtype=torch.int32, device=self.device)
+        if out.numel():
+            class _View:
+                __cuda_array_interface__ = {"shape": shape, "typestr": "<i4", "data": (ptr, False), "version": 3}
+            out.copy_(torch.as_tensor(_View(), device=self.device))
+        return out
+
+    def coarse_coords(self) -> torch.Tensor:
+        """Copy of the coarse coordinates, int32 [n_coarse, 4], sorted."""
+        return self._copy(self._coarse_ptr, (self.n_coarse, 4))
+
+    def parent(self) -> torch.Tensor:
+        """Copy of the coarse row of every input row, int32 [n]."""
+        return self._copy(self._parent_ptr, (self.n,))
+
+    def free(self) -> None:
+        if self.handle:
+            lib.spconv_downsample_free(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass
+
+
+def spconv_downsample_build(coords: torch.Tensor, extent, factor: int = 2, stream=None) -> Downsample:
+    """SparseDownsample(factor) coordinates of int32 [N, 4] CUDA coordinates."""
+    _require()
+    coords = _coords_arg(coords)
+    ext = (ctypes.c_int32 * 3)(*[int(v) for v in extent])
+    handle = ctypes.c_void_p()
+    with torch.cuda.device(coords.device):
+        _check(lib.spconv_downsample_build(coords.data_ptr() if coords.numel() else None, coords.shape[0], ext,
+                                           int(factor), _stream(stream), ctypes.byref(handle)))
+    return Downsample(handle.value, coords.device)
+
+
+def _rows_arg(x: torch.Tensor, rows: int, device, what: str) -> torch.Tensor:
+    if x.dtype not in _DTYPES or not x.is_cuda or x.device != device or x.dim() != 2 or x.shape[0] != rows:
+        raise ValueError(f"{what} must be a float32 or bfloat16 CUDA tensor [{rows}, C] on {device}")
+    return x.contiguous()
+
+
+def spconv_downsample_amax(ds: Downsample, x: torch.Tensor, out: torch.Tensor | None = None,
+                           stream=None) -> torch.Tensor:
+    """Max pooling of x [n, C] onto the coarse voxels -> [n_coarse, C]."""
+    _require()
+    x = _rows_arg(x, ds.n, ds.device, "x")
+    if out is None:
+        out = torch.empty((ds.n_coarse, x.shape[1]), dtype=x.dtype, device=x.device)
+    elif out.shape != (ds.n_coarse, x.shape[1]) or out.dtype != x.dtype or not out.is_contiguous() \
+            or out.device != x.device:
+        raise ValueError("out must be a contiguous [n_coarse, C] tensor like x")
+    if ds.n:
+        with torch.cuda.device(x.device):
+            _check(lib.spconv_downsample_amax(ds.handle, _DTYPES[x.dtype], x.data_ptr(), x.shape[1], out.data_ptr(),
+                                              _stream(stream)))
+    return out
+
+
+def spconv_upsample(ds: Downsample, x_coarse: torch.Tensor, out: torch.Tensor | None = None,
+                    stream=None) -> torch.Tensor:
+    """Coarse features [n_coarse, C] back onto the downsample's input voxels -> [n, C]."""
+    _require()
+    x_coarse = _rows_arg(x_coarse, ds.n_coarse, ds.device, "x_coarse")
+    if out is None:
+        out = torch.empty((ds.n, x_coarse.shape[1]), dtype=x_coarse.dtype, device=x_coarse.device)
+    elif out.shape != (ds.n, x_coarse.shape[1]) or out.dtype != x_coarse.dtype or not out.is_contiguous() \
+            or out.device != x_coarse.device:
+        raise ValueError("out must be a contiguous [n, C] tensor like x_coarse")
+    if ds.n:
+        with torch.cuda.device(x_coarse.device):
+            _check(lib.spconv_upsample(ds.handle, _DTYPES[x_coarse.dtype], x_coarse.data_ptr(), x_coarse.shape[1],
+                                       out.data_ptr(), _stream(stream)))
+    return out
+
+
+def spconv_subdivide(coords: torch.Tensor, extent, x: torch.Tensor | None = None,
+                     stream=None) -> tuple[torch.Tensor, torch.Tensor | None]:
+    """SparseSubdivide: int32 [N, 4] coordinates (and optional features [N, C]) ->
+    the 8 N children (coordinates [8N, 4], features [8N, C]) on the grid 2 * extent."""
+    _require()
+    coords = _coords_arg(coords)
+    n = coords.shape[0]
+    ext = (ctypes.c_int32 * 3)(*[int(v) for v in extent])
+    coords_out = torch.empty((8 * n, 4), dtype=torch.int32, device=coords.device)
+    x_out = None
+    if x is not None:
+        x = _rows_arg(x, n, coords.device, "x")
+        x_out = torch.empty((8 * n, x.shape[1]), dtype=x.dtype, device=x.device)
+    with torch.cuda.device(coords.device):
+        _check(lib.spconv_subdivide(coords.data_ptr() if n else None, n, ext,
+                                    _DTYPES[x.dtype] if x is not None else 0,
+                                    x.data_ptr() if x is not None and n else None,
+                                    x.shape[1] if x is not None else 0, coords_out.data_ptr() if n else None,
+                                    x_out.data_ptr() if x_out is not None and n else None, _stream(stream)))
+    return coords_out, x_out
+
+
 def spconv_debug_set_table_slots(slots: int) -> None:
     _require()
     _check(lib.spconv_debug_set_table_slots(int(slots)))
@@ -266,6 +413,8 @@ def spconv_debug_set_ring_depths(a_slots: int, b_units: int) -> None:
 __all__ = ["OK", "INVALID_ARG", "UNSUPPORTED", "COORD_RANGE", "DUPLICATE", "TABLE_FULL", "OOM", "CUDA_ERROR",
            "TIMEOUT", "SubmMap", "SpconvError", "spconv_build_map", "spconv_subm_forward", "spconv_free",
            "spconv_debug_set_table_slots", "spconv_debug_set_tile_rows", "spconv_debug_set_ring_depths",
-           "spconv_build_neighbor_map_noalloc", "lib",
+           "spconv_build_neighbor_map_noalloc", "lib", "Downsample", "spconv_downsample_build",
+           "spconv_downsample_amax", "spconv_upsample", "spconv_subdivide", "MAP_DEFAULT", "MAP_FLIP_KERNEL",
+           "MAP_SORTED_KEYS",
            "LIB_PATH", "EXPORTED",
            "ALGO_AUTO", "ALGO_SIMT", "ALGO_TCGEN05", "KERNEL_SIMT", "KERNEL_TCGEN05", "KERNEL_NAMES"]

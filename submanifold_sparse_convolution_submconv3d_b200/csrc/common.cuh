@@ -86,6 +86,7 @@ inline int choose_win_rows(int64_t n, int num_sms) {
 struct MapData {
     int64_t n = 0;
     int32_t kernel_size = 3;
+    uint32_t flags = 0;            // spconv_map_flags_t bits the map was built with
     int32_t extent[3] = {0, 0, 0};
     int64_t pairs = 0;
     int32_t* nbr = nullptr;        // device [n, 27] (kernel size 3), else null
@@ -119,12 +120,29 @@ constexpr int kSchedSlots = 64;
 // Sets the calling thread's message returned by spconv_last_error().
 void set_last_error(const std::string& msg);
 
+// Options of the map build.  flip: gather p - d_k instead of p + d_k.  sorted:
+// build the dictionary by radix-sorting the packed keys (skeys[0..1], svals[0..1]:
+// n elements each; hist: radix_hist_words(n) words) and probe it by binary search
+// instead of the hash table (table and slots unused).
+struct MapBuildOpts {
+    bool flip = false;
+    bool sorted = false;
+    uint64_t* skeys[2] = {nullptr, nullptr};
+    int32_t* svals[2] = {nullptr, nullptr};
+    uint32_t* hist = nullptr;
+};
+
+// Key bits of the sorted dictionary for an extent: 16 batch bits plus, per axis,
+// the bits of extent - 1.
+int sorted_key_bits(const int32_t extent[3]);
+
 // Launchers (each returns cudaSuccess or the first CUDA error).
-// Pack + validate + insert, then (kernel size 3) probe into the dense map `nbr`
-// and, when `keys` is not null, the rows' sort keys (Gray rank of the neighbour mask).
+// Pack + validate + build the dictionary, then (kernel size 3) probe into the
+// dense map `nbr` and, when `keys` is not null, the rows' sort keys (Gray rank of
+// the neighbour mask).
 cudaError_t launch_build_map(const int32_t* coords, int64_t n, const int32_t extent[3], int32_t kernel_size,
                              unsigned long long* table, uint64_t slots, int32_t* nbr, uint32_t* keys,
-                             BuildFlags* flags, cudaStream_t stream);
+                             BuildFlags* flags, cudaStream_t stream, const MapBuildOpts& opts = MapBuildOpts());
 
 // Stable radix sort of (key, value) pairs by the low key_bits bits: keys[0] holds
 // the input keys and vals_in the input values (null: the element indices);
@@ -133,6 +151,8 @@ cudaError_t launch_build_map(const int32_t* coords, int64_t n, const int32_t ext
 int64_t radix_hist_words(int64_t n);
 cudaError_t radix_sort_pairs(uint32_t* keys[2], const int32_t* vals_in, int32_t* vals[2], int64_t n, int key_bits,
                              uint32_t* hist, int* which, cudaStream_t stream);
+cudaError_t radix_sort_pairs64(uint64_t* keys[2], const int32_t* vals_in, int32_t* vals[2], int64_t n, int key_bits,
+                               uint32_t* hist, int* which, cudaStream_t stream);
 
 // Window-kernel metadata from the dense map and the sorted rows.
 cudaError_t launch_win_meta(const int32_t* nbr, const int32_t* sorted_rows, int64_t n, int rows, int64_t tiles,
