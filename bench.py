@@ -13,9 +13,13 @@ output copied back.
 
 per_config times the other workloads' layers the same way (one captured layer,
 L2 flushed before each replay), each against its own roofline, and the 512^3
-shell workload end to end (map build + layer).
+shell workload end to end (map build + layer) with both map dictionaries.
+resample_chain times downsample -> conv -> subdivide -> conv on the 256^3 shells,
+a new map built for every new coordinate set.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py --profile-layer WORKLOAD        # small fixed runs for ncu
+    python bench.py --profile-build WORKLOAD:hash|sorted|auto
 
 Under torchrun each rank runs the same workload on its own GPU (replicas; the
 layer has no exchange step), times are the max over ranks, value is the sum.
@@ -67,8 +71,9 @@ PER_CONFIG = (  # (workload, layer index, label)
 # sources it was taken on: reported as null once their hash changes.
 PROFILED_TRAFFIC = {
     "kernel": "k_subm_win<128,128>",
-    "bytes": None,
-    "sources_sha256": None,
+    # profiles/k_subm_win_uniform128.md: 65,435,648 B read + 19,799,808 B written
+    "bytes": 85235456,
+    "sources_sha256": "60b1e989673e89c67881bf20fc0e55bbd44ad81182ee37db34c0e608589b75a6",
 }
 KERNEL_SOURCES = ("forward_win.cu", "sm100.cuh", "common.cuh")
 
@@ -297,8 +302,8 @@ def run_per_config(sp, dev, flush, reps: int, hbm: float, tflops: float, cpu: bo
         del g
         m.free()
         if name == "large":
-            # end to end on the GPU: map build (hash, probe, row sort, tile metadata;
-            # one stream synchronisation inside) then the layer, host-timed
+            # end to end on the GPU: map build (dictionary, probe, row sort, tile
+            # metadata; one stream synchronisation inside) then the layer, host-timed
             e2e, builds, fwds = [], [], []
             for _ in range(4):
                 flush.fill_(1.0)
@@ -316,12 +321,122 @@ def run_per_config(sp, dev, flush, reps: int, hbm: float, tflops: float, cpu: bo
             e["end_to_end"] = {"ms_median": statistics.median(e2e[1:]), "map_build_ms_median": statistics.median(builds[1:]),
                                "forward_ms_median": statistics.median(fwds[1:]),
                                "includes": "map build (one stream synchronisation) + one layer, host-timed, L2 flushed"}
+            # the two dictionaries of the map build, each forced (bit-identical maps)
+            e["map_build_ms_by_dictionary"] = {
+                "hash_table": build_ms_median(sp, coords_d, wl.grid, flush, sorted_keys=False),
+                "sorted_keys": build_ms_median(sp, coords_d, wl.grid, flush, sorted_keys=True),
+                "library_choice": "sorted_keys" if wl.n >= 1 << 20 else "hash_table"}
         if cpu:
             e["cpu_baseline"] = cpu_oracle_sample(wl, layer, target_s=1.5)
         results.append(e)
         del x, w, b, o, coords_d
         torch.cuda.empty_cache()
     return results
+
+def build_ms_median(sp, coords_d, grid, flush, sorted_keys=None, reps: int = 5) -> float:
+    """Host-timed map build (one synchronisation inside), L2 flushed first; median
+    of reps after one untimed build."""
+    import torch
+    ms = []
+    for i in range(reps + 1):
+        flush.fill_(1.0)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        mm = sp.spconv_build_map(coords_d, grid, 3, sorted_keys=sorted_keys)
+        dt = (time.perf_counter() - t0) * 1e3
+        mm.free()
+        if i:
+            ms.append(dt)
+    return statistics.median(ms)
+
+
+def run_resample_chain(sp, dev, flush, reps: int = 5) -> dict:
+    """The coordinate-changing ops around the convolution on the 256^3 shells,
+    one pass = SparseDownsample(2) coordinates + amax pooling, a map build on the
+    coarse set, a 64 -> 64 layer there, SparseSubdivide back to the fine grid, a
+    map build on the subdivided set and a layer there.  Host-timed per stage with
+    a synchronisation after each (the builds synchronise anyway)."""
+    import torch
+    wl = workloads.make_workload("shells", 0)
+    coords_d = torch.from_numpy(wl.coords).to(dev)
+    x = torch.from_numpy(wl.x).to(dev, torch.bfloat16)
+    w = torch.from_numpy(wl.layers[0].w).to(dev, torch.bfloat16)
+    b = torch.from_numpy(wl.layers[0].bias).to(dev, torch.bfloat16)
+    stages = ("downsample_build", "amax", "coarse_map_build", "coarse_layer", "subdivide", "fine_map_build",
+              "fine_layer")
+    times = {k: [] for k in stages}
+    sizes = {}
+    for it in range(reps + 1):
+        flush.fill_(1.0)
+        torch.cuda.synchronize()
+        t = [time.perf_counter()]
+
+        def mark():
+            torch.cuda.synchronize()
+            t.append(time.perf_counter())
+        ds = sp.spconv_downsample_build(coords_d, wl.grid, 2)
+        mark()
+        pooled = sp.spconv_downsample_amax(ds, x)
+        mark()
+        cc = ds.coarse_coords()
+        cm = sp.spconv_build_map(cc, ds.coarse_extent, 3)
+        mark()
+        y = sp.spconv_subm_forward(cm, pooled, w, b)
+        mark()
+        fc, fx = sp.spconv_subdivide(cc, ds.coarse_extent, y)
+        mark()
+        fext = tuple(2 * e for e in ds.coarse_extent)
+        fm = sp.spconv_build_map(fc, fext, 3)
+        mark()
+        z = sp.spconv_subm_forward(fm, fx, w, b)
+        mark()
+        cm.check()
+        fm.check()
+        sizes = {"fine_voxels": wl.n, "coarse_voxels": ds.n_coarse, "subdivided_voxels": int(fc.shape[0])}
+        cm.free()
+        fm.free()
+        ds.free()
+        del pooled, y, fx, z, cc, fc
+        if it:
+            for k, i in zip(stages, range(len(stages))):
+                times[k].append((t[i + 1] - t[i]) * 1e3)
+    med = {k: statistics.median(v) for k, v in times.items()}
+    return {"config": "shells 256^3: downsample(2) -> conv -> subdivide -> conv (64 ch, bf16)", **sizes,
+            "stage_ms_median": med, "total_ms_median": sum(med.values()),
+            "timing": "host clock, a synchronisation after every stage, L2 flushed before each pass"}
+
+
+def run_profile_mode(args) -> None:
+    """A small fixed run for ncu captures (committed, so profile summaries can name
+    their command): --profile-layer NAME runs the map build and three launches of
+    the workload's first layer; --profile-build NAME:DICT runs three map builds with
+    the dictionary DICT (hash, sorted or auto)."""
+    import torch
+
+    import submanifold_sparse_convolution_submconv3d_b200 as sp
+    dev = torch.device("cuda", 0)
+    if args.profile_layer:
+        wl = workloads.make_workload(args.profile_layer, 0, n_layers=1)
+        m = sp.spconv_build_map(torch.from_numpy(wl.coords).to(dev), wl.grid, wl.layers[0].kernel_size)
+        x = torch.from_numpy(wl.x).to(dev, torch.bfloat16)
+        w = torch.from_numpy(wl.layers[0].w).to(dev, torch.bfloat16)
+        b = torch.from_numpy(wl.layers[0].bias).to(dev, torch.bfloat16)
+        out = torch.empty((wl.n, w.shape[2]), dtype=torch.bfloat16, device=dev)
+        for _ in range(3):
+            sp.spconv_subm_forward(m, x, w, b, out=out)
+        torch.cuda.synchronize()
+        m.check()
+        m.free()
+    else:
+        name, _, dic = args.profile_build.partition(":")
+        wl = workloads.make_workload(name, 0, n_layers=1)
+        c = torch.from_numpy(wl.coords).to(dev)
+        sk = {"hash": False, "sorted": True}.get(dic)
+        for _ in range(3):
+            sp.spconv_build_map(c, wl.grid, 3, sorted_keys=sk).free()
+        torch.cuda.synchronize()
+    print(json.dumps({"profile_run": "ok"}))
+
 
 def run_reference(args, rank: int, world: int) -> None:
     """The reference arm: the CPU oracle as it stands on the host cores (rank 0 only),
@@ -447,8 +562,10 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     hbm, tf_burst, tf_sust, peak_kind = _peaks()
     layer_s = statistics.median(step_ms) / LAYERS / 1e3
     per_config = None
+    resample = None
     if world == 1 and not args.no_per_config:
         per_config = run_per_config(sp, dev, flush, 10, hbm, tf_burst, cpu=not args.no_cpu_baseline)
+        resample = run_resample_chain(sp, dev, flush)
     if rank != 0:
         return
     rf = roofline(n, pairs, cin, cout, 27, layer_s, hbm, tf_burst)
@@ -489,6 +606,8 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     }
     if per_config is not None:
         line["per_config"] = per_config
+    if resample is not None:
+        line["resample_chain"] = resample
     if world == 1 and not args.no_cpu_baseline:
         wl1 = workloads.make_workload(WORKLOAD, 0, n_layers=1)
         line["cpu_baseline"] = cpu_oracle_sample(wl1, wl1.layers[0], 10.0)
@@ -503,7 +622,12 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true")
+    ap.add_argument("--profile-layer", default=None, help="workload: map build + 3 launches of its first layer (ncu)")
+    ap.add_argument("--profile-build", default=None, help="workload:hash|sorted|auto: 3 map builds (ncu)")
     args = ap.parse_args()
+    if args.profile_layer or args.profile_build:
+        run_profile_mode(args)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
