@@ -35,10 +35,12 @@
 //   warps 2-5   gather producers (B operand).  A tile's index stream arrives in
 //               shared memory by one bulk copy, a tile ahead, into one of two
 //               buffers.  The B ring is cut into units of 64 rows; a job takes
-//               ceil(N / 64) consecutive units (never wrapping); all four warps
-//               fill every unit, 16 rows each, with 16-byte cp.async copies (zero
-//               fill for holes) into the swizzled K-major layout the MMA reads, so
-//               each unit's uses are filled and drained strictly in turn
+//               ceil(N / 64) consecutive units (never wrapping); each unit
+//               belongs to a fixed group of gather warps (all four for
+//               128-channel chunks, two otherwise), which fill every use of it
+//               with 16-byte cp.async copies (zero fill for holes) into the swizzled
+//               K-major layout the MMA reads, so each unit's uses are filled and
+//               drained strictly in turn
 //   warps 6-13  epilogue: two warps per TMEM lane quarter, alternate 32-column
 //               chunks (warp w covers lanes 32 (w % 4) .. +31, the hardware's rule
 //               for TMEM access): accumulator + bias -> bf16, staged in shared memory, then
@@ -99,15 +101,11 @@ struct WinLayout {
     static constexpr int kARB = kAtomElems * 2;                // atom row bytes: 128, 64 or 32
     static constexpr int kUnitAtomBytes = kUnitRows * kARB;    // a multiple of the swizzle repeat
     static constexpr int kUnitBytes = kAtoms * kUnitAtomBytes;
-    static constexpr int kThreadsPerRow = KC * 2 / 16;         // 16-byte chunks of one row's chunk
-    static constexpr int kWarpRows = 32 / kThreadsPerRow;      // rows one warp instruction covers
-    static constexpr int kSliceRows = kUnitRows / kGatherWarps;  // rows of a unit one gather warp fills
-    // passes of one warp instruction over a slice; when one instruction covers more
-    // rows than a slice holds, the lanes past the slice stay idle
-    static constexpr int kPasses = (kSliceRows + kWarpRows - 1) / kWarpRows;
-    static_assert(kSliceRows % kWarpRows == 0 || kWarpRows % kSliceRows == 0, "slices and passes must align");
-    static constexpr int kChunksPerAtom = kARB / 16;
-    static constexpr uint32_t kSwz = kARB / 16 - 1;
+    // Gather warps that fill one unit together (its rows split between them): 4
+    // for 128-channel chunks, whose units are few and whose jobs wait on their fill
+    // latency; 2 for narrower chunks, whose deeper rings gain from two units
+    // filled at once (measured on B200: 1, 2 and 4 warps per unit).
+    static constexpr int kFillWarps = KC >= 128 ? 4 : 2;
     static constexpr uint32_t kBLayout = kARB == 128 ? 2u : (kARB == 64 ? 4u : 6u);
     static constexpr uint32_t kBSbo = 8 * kARB;
     static constexpr int kStepsPerAtom = kAtomElems / 16;
@@ -246,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(emptyA0 + 8 * s, 1);
         }
         for (int u = 0; u < UB; ++u) {
-            mbar_init(fullB0 + 8 * u, 32 * kGatherWarps);  // every lane of every gather warp
+            mbar_init(fullB0 + 8 * u, 32 * L::kFillWarps);  // every lane of the unit's filling warps
             mbar_init(emptyB0 + 8 * u, 1);
         }
         for (int b = 0; b < kAccBufs; ++b) {
@@ -505,14 +503,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (warp < kWarpEpi0) {
         // ------------------------------------------------ gather producers
-        // Gather warp g fills rows [16 g, 16 g + 16) of every unit.  Lane l copies
-        // 16-byte chunk l % kThreadsPerRow of rows l / kThreadsPerRow + kWarpRows *
-        // pass.  The source rows of all passes are read first (rows past the job
-        // read as holes, so no pass branches), then every pass issues its copy.
+        // The gather warps form kGroups groups of kFillWarps; unit u belongs to
+        // group u % kGroups, whose warps fill every use of it (warp sub of the group
+        // its slice of kSliceRows rows), so kGroups units fill at once.  Every use
+        // of a unit is thus waited for and filled by the same warps, in order: no
+        // warp reaches a unit's next use before the previous one was released,
+        // which the phase-parity wait could not tell apart from the use before it.
+        // Lane l copies 16-byte chunk l % kThreadsPerRow of rows
+        // l / kThreadsPerRow + kWarpRows * pass of its slice.
+        constexpr int kThreadsPerRow = KC * 2 / 16;                // 16-byte chunks of one row's chunk
+        constexpr int kWarpRows = 32 / kThreadsPerRow;             // rows one warp instruction covers
+        constexpr int kSliceRows = kUnitRows / L::kFillWarps;      // rows of a unit one warp fills
+        constexpr int kGroups = kGatherWarps / L::kFillWarps;      // groups of warps that share units
+        // passes of one warp instruction over its slice, taken kBatch at a time; when
+        // one instruction covers more rows than a slice holds, lanes past it idle
+        constexpr int kPasses = kSliceRows >= kWarpRows ? kSliceRows / kWarpRows : 1;
+        constexpr int kBatch = kPasses < 8 ? kPasses : 8;
+        static_assert(kSliceRows % kWarpRows == 0 || kWarpRows % kSliceRows == 0, "slices and passes must align");
+        static_assert(kPasses % kBatch == 0, "batches must tile the passes");
+        constexpr int kChunksPerAtom = L::kARB / 16;
+        constexpr uint32_t kSwz = L::kARB / 16 - 1;
         const int g = warp - kWarpGather0;
-        const int q = lane % L::kThreadsPerRow;
-        const int prow = lane / L::kThreadsPerRow;
-        const int atom = q / L::kChunksPerAtom, qa = q % L::kChunksPerAtom;
+        const int grp = g / L::kFillWarps, sub = g % L::kFillWarps;  // unit group, slice within a unit
+        const int q = lane % kThreadsPerRow;
+        const int prow = lane / kThreadsPerRow;
+        const int atom = q / kChunksPerAtom, qa = q % kChunksPerAtom;
         const bool issuer = g == 0 && p.idx_stream != nullptr;  // fetches the index streams
         int ucur = 0;
         uint32_t bph = 0;
@@ -572,33 +587,38 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __nv_bfloat16* xc = p.x + c * KC + q * 8;
                     for (int qq = 0; qq < m; ++qq) {
                         const int unit = u0 + qq;
+                        if (unit % kGroups != grp) continue;  // another group's unit
                         if (!warp_wait_bar<kSleepProducer>(emptyB0 + 8 * unit, ((bph >> unit) & 1u) ^ 1u, abort_flag,
                                                            p.err)) {
                             aborted = true;
                             break;
                         }
-                        const int jr0 = qq * kUnitRows + g * L::kSliceRows;  // first job row of this slice
-                        int src[L::kPasses];
-#pragma unroll
-                        for (int pp = 0; pp < L::kPasses; ++pp) {
-                            const int r = jr0 + prow + pp * L::kWarpRows;  // job row
-                            if (p.idx_stream) {
-                                const int v = ibuf[joff + r];
-                                src[pp] = r < ncols ? v : -1;
-                            } else {
-                                const int64_t rr = r0 + r;
-                                src[pp] = r < ncols && rr < p.n ? (int)rr : -1;
-                            }
-                        }
                         const uint32_t ubase = smem_addr(b_ring) + (uint32_t)(atom * UB * L::kUnitAtomBytes) +
                                                (uint32_t)(unit * L::kUnitAtomBytes);
+                        // kBatch passes at a time: their source rows first (rows past the
+                        // job read as holes, so no pass branches), then their copies
+#pragma unroll 1
+                        for (int p0 = 0; p0 < kPasses; p0 += kBatch) {
+                            int src[kBatch];
 #pragma unroll
-                        for (int pp = 0; pp < L::kPasses; ++pp) {
-                            if (L::kWarpRows > L::kSliceRows && prow >= L::kSliceRows) continue;
-                            const uint32_t lin =
-                                (uint32_t)((g * L::kSliceRows + prow + pp * L::kWarpRows) * L::kARB + qa * 16);
-                            cp_async_16(ubase + (lin ^ (((lin >> 7) & L::kSwz) << 4)),
-                                        xc + (int64_t)(src[pp] >= 0 ? src[pp] : 0) * p.cin, src[pp] >= 0 ? 16u : 0u);
+                            for (int pp = 0; pp < kBatch; ++pp) {
+                                const int r = qq * kUnitRows + sub * kSliceRows + prow + (p0 + pp) * kWarpRows;
+                                if (p.idx_stream) {
+                                    const int v = ibuf[joff + r];
+                                    src[pp] = r < ncols ? v : -1;
+                                } else {
+                                    const int64_t rr = r0 + r;
+                                    src[pp] = r < ncols && rr < p.n ? (int)rr : -1;
+                                }
+                            }
+#pragma unroll
+                            for (int pp = 0; pp < kBatch; ++pp) {
+                                if (kWarpRows > kSliceRows && prow >= kSliceRows) continue;
+                                const uint32_t lin =
+                                    (uint32_t)((sub * kSliceRows + prow + (p0 + pp) * kWarpRows) * L::kARB + qa * 16);
+                                cp_async_16(ubase + (lin ^ (((lin >> 7) & kSwz) << 4)),
+                                            xc + (int64_t)(src[pp] >= 0 ? src[pp] : 0) * p.cin, src[pp] >= 0 ? 16u : 0u);
+                            }
                         }
                         cp_async_mbar_arrive_noinc(fullB0 + 8 * unit);
                     }
