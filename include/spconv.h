@@ -16,7 +16,7 @@
  * columns 1, 2, 3); the centre offset is k = 13.
  *
  * The neighbour map is built once per coordinate set and cached in a handle,
- * as the pages' "cached device index" does (lato.2_mrp_mlx README, "Fleet
+ * as the pages cache their prepared device index (lato.2_mrp_mlx README, "Fleet
  * benchmark"); the map build is the step the same section names as dominant
  * whenever coordinates change.  The trellis-mac article (section on sparse 3D
  * convolution, gather-scatter) builds a hash map of active voxel coordinates
@@ -112,10 +112,10 @@ SPCONV_API spconv_status_t spconv_build_map(const int32_t* coords, int64_t n, co
  *                           one behind its --flip-kernel switch.  The map is the
  *                           default map with offsets k and 26 - k exchanged.
  *   SPCONV_MAP_SORTED_KEYS  build the coordinate dictionary by radix-sorting the
- *                           packed keys and find every neighbour by binary search,
- *                           the "sorted-key indice map" the lato.2_mrp_mlx README
- *                           (table of upstream equivalents) names for its port,
- *                           instead of the hash table.  Same map, bit for bit.
+ *                           packed keys and find every neighbour by binary search
+ *                           -- the sorted-key index map that the lato.2_mrp_mlx
+ *                           README's table of upstream equivalents gives for its
+ *                           port -- instead of the hash table.  Same map, bit for bit.
  *                           Needs 16 + sum over axes of ceil(log2(extent)) <= 62
  *                           (SPCONV_ERR_UNSUPPORTED otherwise); never reports
  *                           SPCONV_ERR_TABLE_FULL.

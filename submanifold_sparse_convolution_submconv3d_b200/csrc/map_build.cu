@@ -7,9 +7,9 @@
 // caches the resulting index per coordinate set.  Two dictionaries are built
 // here, both writing the same dense [n, 27] index map with -1 holes:
 //   - an open-addressing hash table over 64-bit packed keys (the default);
-//   - the sorted-key form the lato.2_mrp_mlx README's table of upstream
-//     equivalents names for its own port ("a sorted-key indice map"): the packed
-//     keys radix-sorted with their rows, each neighbour found by binary search.
+//   - the sorted-key index map that the lato.2_mrp_mlx README's table of
+//     upstream equivalents gives for its own port: the packed keys radix-sorted
+//     with their rows, each neighbour found by binary search.
 // Orientation: the map gathers p + d_k (cross-correlation, as the README's
 // "Correctness" section says the port implements) or, with the flip option,
 // p - d_k (the alternative the same section leaves open and its --flip-kernel
