@@ -50,6 +50,7 @@
 // in the map's error word, stops issuing work, lets copies in flight land, waits
 // (bounded) for its MMAs and frees its TMEM before returning.
 #include <atomic>
+#include <cstring>
 #include <mutex>
 #include <vector>
 
@@ -146,6 +147,7 @@ struct WinParams {
     unsigned int* err;
     int sa, ub;                 // weight-ring slots, B-ring units
     int idx_buf_elems;          // int32 entries of one tile index buffer
+    int rows_tma;               // kernel size 1 with n >= 64: B units loaded as 64-row TMA tiles
 };
 
 // Waiting policy.  A waiting thread polls the barrier; while the phase is not
@@ -210,7 +212,7 @@ __device__ __forceinline__ const uint32_t* slot_rec(const uint8_t* slot) {
 
 template <int BM, int KC>
 __global__ void __launch_bounds__(kThreads, 1)
-    k_subm_win(const __grid_constant__ CUtensorMap wmap, const WinParams p) {
+    k_subm_win(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap, const WinParams p) {
     using L = WinLayout<BM, KC>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -244,7 +246,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(emptyA0 + 8 * s, 1);
         }
         for (int u = 0; u < UB; ++u) {
-            mbar_init(fullB0 + 8 * u, 32 * L::kFillWarps);  // every lane of the unit's filling warps
+            // cp.async fill: every lane of the unit's filling warps; TMA tile: the
+            // issuing thread's expect-tx arrival, then the bytes
+            mbar_init(fullB0 + 8 * u, p.rows_tma ? 1 : 32 * L::kFillWarps);
             mbar_init(emptyB0 + 8 * u, 1);
         }
         for (int b = 0; b < kAccBufs; ++b) {
@@ -588,6 +592,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int qq = 0; qq < m; ++qq) {
                         const int unit = u0 + qq;
                         if (unit % kGroups != grp) continue;  // another group's unit
+                        if (p.rows_tma) {
+                            // kernel size 1: the job's rows are consecutive input rows, so
+                            // the unit is one 64-row tile per channel atom (rows past n
+                            // read as zeros); the group's first warp loads it
+                            if (sub != 0) continue;
+                            if (!warp_wait_bar<kSleepProducer>(emptyB0 + 8 * unit, ((bph >> unit) & 1u) ^ 1u,
+                                                               abort_flag, p.err)) {
+                                aborted = true;
+                                break;
+                            }
+                            if (lane == 0) {
+                                const uint32_t full = fullB0 + 8 * unit;
+                                mbar_arrive_expect_tx(full, (uint32_t)L::kUnitBytes);
+#pragma unroll
+                                for (int at = 0; at < L::kAtoms; ++at)
+                                    tma_load_2d(smem_addr(b_ring) + (uint32_t)((at * UB + unit) * L::kUnitAtomBytes),
+                                                &xmap, c * KC + at * L::kAtomElems, (int)(r0 + qq * kUnitRows), full);
+                            }
+                            __syncwarp();
+                            continue;
+                        }
                         if (!warp_wait_bar<kSleepProducer>(emptyB0 + 8 * unit, ((bph >> unit) & 1u) ^ 1u, abort_flag,
                                                            p.err)) {
                             aborted = true;
@@ -632,7 +657,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(tileE0 + 8 * s);
             }
         }
-        if (issuer && aborted && lane == 0) __nanosleep(200000);  // the index copy in flight lands first
+        // copies in flight (an index stream, row tiles) land before the CTA exits
+        if ((issuer || p.rows_tma) && aborted && lane == 0) __nanosleep(200000);
         cp_async_wait_all();
     } else if (warp < kWarpEpi0 + kEpiWarps) {
         // ------------------------------------------------ epilogue
@@ -790,6 +816,27 @@ spconv_status_t launch(const MapData& m, const void* x, int cin, const void* w, 
         *ce = cudaErrorInvalidValue;
         return SPCONV_ERR_CUDA;
     }
+    // Features [n, cin] as 64-row tiles of one channel atom, for kernel size 1 (no
+    // gather: a job's rows are consecutive); swizzled like the B ring.  Encoded
+    // only when used, and then n >= 64 (one tile at most as tall as the tensor).
+    CUtensorMap xmap;
+    memset(&xmap, 0, sizeof(xmap));
+    const bool rows_tma = kvol == 1 && m.n >= kUnitRows;
+    if (rows_tma) {
+        const cuuint64_t xdims[2] = {(cuuint64_t)cin, (cuuint64_t)m.n};
+        const cuuint64_t xstrides[1] = {(cuuint64_t)cin * 2};
+        const cuuint32_t xbox[2] = {(cuuint32_t)L::kAtomElems, (cuuint32_t)kUnitRows};
+        const CUtensorMapSwizzle xswz = L::kARB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                                        : (L::kARB == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                                         : CU_TENSOR_MAP_SWIZZLE_32B);
+        r = enc(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), xdims, xstrides, xbox, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, xswz, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) {
+            *ce = cudaErrorInvalidValue;
+            return SPCONV_ERR_CUDA;
+        }
+    }
     const int need_smem = L::smem_bytes(sa, ub, max_cols);
     const int smem = need_smem > kMinSmem ? need_smem : kMinSmem;
     int dev = 0;
@@ -836,9 +883,10 @@ spconv_status_t launch(const MapData& m, const void* x, int cin, const void* w, 
     p.sa = sa;
     p.ub = ub;
     p.idx_buf_elems = L::idx_buf_bytes(max_cols) / 4;
+    p.rows_tma = rows_tma ? 1 : 0;
     const int64_t units = m.win_tiles * p.cblocks;
     const int64_t grid = units < m.num_sms ? units : m.num_sms;
-    k_subm_win<BM, KC><<<(unsigned)grid, kThreads, smem, stream>>>(map, p);
+    k_subm_win<BM, KC><<<(unsigned)grid, kThreads, smem, stream>>>(map, xmap, p);
     *ce = cudaGetLastError();
     return *ce == cudaSuccess ? SPCONV_OK : SPCONV_ERR_CUDA;
 }
