@@ -34,6 +34,16 @@ coarse grid is ceil(extent / factor); "amax" of a block is the largest value,
 with +0 above -0 (the IEEE 754 total order); subdivision lists the children of
 voxel i as rows 8 i + c, c = 4 ox + 2 oy + oz, each carrying voxel i's features.
 
+The fused decoder epilogue (``epilogue``, ``channel_stats``): the pixal3d_mrp_mlx
+README ("Correction to the earlier scope") lists SparseConvNeXtBlock3d and
+SparseResBlockC2S3d among the decoder blocks around the convolution, and the
+lato.2_mrp_mlx README ("Status") lists the activations, norms and SparseResBlock
+of the shared core.  Reading: the convolution's store may apply, in this order,
+an activation to conv + bias (ReLU, SiLU, or GELU with the exact erf), then add a
+residual of the output's shape, and may report per output channel the sum and
+the sum of squares of the stored (rounded) output over all rows, which a
+following LayerNorm / GroupNorm needs.
+
 Pins: every function here is pinned by ``tests/test_oracle_pins.py`` against
 dense brute force, torch's CPU conv3d, closed forms and invariants; none is
 "parity unpinned".
@@ -258,3 +268,43 @@ def downsample_py(coords, factor: int = 2):
         for i in blocks[key]:
             parent[i] = g
     return np.array(keys, dtype=np.int32).reshape(-1, 4), np.array(parent, dtype=np.int32)
+
+
+# ---------------------------------------------------------------------------
+# Fused decoder epilogue: activation, residual add, per-channel statistics.
+# ---------------------------------------------------------------------------
+
+ACTIVATIONS = ("none", "relu", "silu", "gelu")
+
+
+def activation(name: str, y) -> np.ndarray:
+    """The activation applied to conv + bias, in fp64: ReLU max(y, 0); SiLU
+    y * sigmoid(y) = y / (1 + exp(-y)); GELU 0.5 y (1 + erf(y / sqrt 2))."""
+    y = np.asarray(y, dtype=np.float64)
+    if name == "none":
+        return y.copy()
+    if name == "relu":
+        return np.maximum(y, 0.0)
+    if name == "silu":
+        with np.errstate(over="ignore"):
+            return y / (1.0 + np.exp(-y))
+    if name == "gelu":
+        from scipy.special import erf  # a library routine as one step
+        return 0.5 * y * (1.0 + erf(y / np.sqrt(2.0)))
+    raise ValueError(f"unknown activation {name!r}")
+
+
+def epilogue(conv, act: str = "none", residual=None) -> np.ndarray:
+    """The stored value before rounding: act(conv) (+ residual), where conv is the
+    convolution output with its bias (fp64, e.g. from ``forward``)."""
+    y = activation(act, conv)
+    if residual is not None:
+        y = y + np.asarray(residual, dtype=np.float64)
+    return y
+
+
+def channel_stats(out) -> np.ndarray:
+    """[2, C]: per channel the sum and the sum of squares of the stored output over
+    all rows, in fp64 (out holds the stored, rounded values)."""
+    o = np.asarray(out, dtype=np.float64)
+    return np.stack([o.sum(axis=0), (o * o).sum(axis=0)])

@@ -1,5 +1,6 @@
-"""Pins for the oracle's kernel-orientation option and its resampling functions
-(SparseDownsample with amax, its paired SparseUpsample, SparseSubdivide).
+"""Pins for the oracle's kernel-orientation option, its resampling functions
+(SparseDownsample with amax, its paired SparseUpsample, SparseSubdivide) and its
+fused decoder epilogue (activation, residual, per-channel statistics).
 
 Each is checked against something other than the oracle itself: torch's CPU
 conv3d with the kernel mirrored (a true convolution), torch's dense max_pool3d
@@ -7,6 +8,8 @@ and nearest-neighbour interpolate on zero/-inf-filled grids, hand-worked
 examples, the pure-Python twins, and invariants that tie the functions together
 (downsampling a subdivision gives back the original set and features).
 """
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -206,3 +209,59 @@ def test_downsample_inverts_subdivide():
     assert cext == extent
     assert np.array_equal(coarse, coords[order])
     assert np.array_equal(oracle.downsample_amax(parent, coarse.shape[0], xf), x[order])
+
+
+# ------------------------------------------------------------------ epilogue
+
+@pytest.mark.parametrize("act", ["relu", "silu", "gelu"])
+def test_activations_match_torch(act):
+    y = np.concatenate([np.linspace(-12, 12, 2001), [0.0, -0.0, 1e-30, -1e-30, 40.0, -40.0]])
+    got = oracle.activation(act, y)
+    t = torch.from_numpy(y)
+    ref = {"relu": torch.nn.functional.relu, "silu": torch.nn.functional.silu,
+           "gelu": lambda v: torch.nn.functional.gelu(v, approximate="none")}[act](t).numpy()
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-15)
+
+
+def test_activation_hand_values():
+    assert oracle.activation("relu", [-2.0, 3.0]).tolist() == [0.0, 3.0]
+    assert oracle.activation("silu", [0.0])[0] == 0.0
+    assert abs(oracle.activation("silu", [1.0])[0] - 1.0 / (1.0 + math.exp(-1.0))) < 1e-16
+    assert abs(oracle.activation("gelu", [1.0])[0] - 0.8413447460685429) < 1e-15  # 1 * Phi(1)
+    assert oracle.activation("none", [-5.0])[0] == -5.0
+    with pytest.raises(ValueError):
+        oracle.activation("tanh", [0.0])
+
+
+def test_epilogue_order_and_residual():
+    """act applies to conv + bias, then the residual is added: relu(-1) + 5 = 5, not relu(4)."""
+    conv = np.array([[-1.0, 2.0]])
+    res = np.array([[5.0, -3.0]])
+    assert oracle.epilogue(conv, "relu", res).tolist() == [[5.0, -1.0]]
+    assert oracle.epilogue(conv, "none", None).tolist() == [[-1.0, 2.0]]
+
+
+def test_residual_conv_equals_conv_of_identity_tap_plus_conv():
+    """A residual x added to conv(x, W) equals conv(x, W') with W'[13] = W[13] + I
+    (the centre tap sees the voxel itself): an identity of the definition."""
+    rng = np.random.default_rng(22)
+    coords = _random_set(rng, (6, 6, 6), 60)
+    x = rng.standard_normal((60, 4))
+    w = rng.standard_normal((27, 4, 4))
+    nbr = oracle.neighbor_map(coords, (6, 6, 6))
+    lhs = oracle.epilogue(oracle.forward(nbr, x, w), "none", x)
+    w2 = w.copy()
+    w2[13] += np.eye(4)
+    np.testing.assert_allclose(lhs, oracle.forward(nbr, x, w2), rtol=1e-12, atol=1e-12)
+
+
+def test_channel_stats_match_torch_moments():
+    rng = np.random.default_rng(23)
+    out = rng.standard_normal((500, 7))
+    s = oracle.channel_stats(out)
+    t = torch.from_numpy(out)
+    n = out.shape[0]
+    np.testing.assert_allclose(s[0] / n, t.mean(dim=0).numpy(), rtol=1e-12, atol=1e-14)
+    var = s[1] / n - (s[0] / n) ** 2
+    np.testing.assert_allclose(var, t.var(dim=0, unbiased=False).numpy(), rtol=1e-9, atol=1e-12)
+    assert oracle.channel_stats(np.array([[1.0, -2.0], [3.0, 4.0]])).tolist() == [[4.0, 2.0], [10.0, 20.0]]
