@@ -333,6 +333,42 @@ def run_per_config(sp, dev, flush, reps: int, hbm: float, tflops: float, cpu: bo
         torch.cuda.empty_cache()
     return results
 
+def run_fused_epilogue(sp, dev, flush, reps: int, hbm: float, tflops: float) -> dict:
+    """The 128^3 layer with the fused decoder epilogue (SiLU of conv + bias, a
+    residual add, per-channel sums for a following norm), next to the plain layer
+    in the same run; the roofline adds the residual's read."""
+    import torch
+    wl = workloads.make_workload(WORKLOAD, 0, n_layers=1)
+    layer = wl.layers[0]
+    m = sp.spconv_build_map(torch.from_numpy(wl.coords).to(dev), wl.grid, 3)
+    x = torch.from_numpy(wl.x).to(dev, torch.bfloat16)
+    w = torch.from_numpy(layer.w).to(dev, torch.bfloat16)
+    b = torch.from_numpy(layer.bias).to(dev, torch.bfloat16)
+    res = torch.from_numpy(workloads.round_to_bf16(np.random.default_rng(7).standard_normal(
+        (wl.n, 128), dtype=np.float32))).to(dev, torch.bfloat16)
+    o = torch.empty((wl.n, 128), dtype=torch.bfloat16, device=dev)
+    stats = torch.empty((2, 128), dtype=torch.float32, device=dev)
+    times = {}
+    for name, fn in (("plain", lambda: sp.spconv_subm_forward(m, x, w, b, out=o)),
+                     ("fused", lambda: sp.spconv_subm_forward(m, x, w, b, out=o, act="silu", residual=res,
+                                                              stats=stats))):
+        g = capture_graph(fn)
+        for _ in range(3):
+            g.replay()
+        times[name] = statistics.median(time_replays(g, reps, flush)) / 1e3
+        del g
+    m.check()
+    rf = roofline(wl.n, m.pairs, 128, 128, 27, times["fused"], hbm, tflops)
+    extra = wl.n * 128 * 2 + 2 * 128 * 4  # residual read, statistics written
+    m.free()
+    return {"config": "uniform k=3 128->128 + SiLU + residual + channel sums (fused epilogue)",
+            "layer_us_median": times["fused"] * 1e6, "plain_layer_us_median": times["plain"] * 1e6,
+            "kernel": tc_kernel_name(128, 128) + " (fused instantiation)",
+            "roofline": {**rf, "algorithmic_bytes": rf["algorithmic_bytes"] + extra,
+                         "t_roof_us": max((rf["algorithmic_bytes"] + extra) / (hbm * 1e9),
+                                          rf["useful_flops"] / (tflops * 1e12)) * 1e6}}
+
+
 def build_ms_median(sp, coords_d, grid, flush, sorted_keys=None, reps: int = 5) -> float:
     """Host-timed map build (one synchronisation inside), L2 flushed first; median
     of reps after one untimed build."""
@@ -565,6 +601,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     resample = None
     if world == 1 and not args.no_per_config:
         per_config = run_per_config(sp, dev, flush, 10, hbm, tf_burst, cpu=not args.no_cpu_baseline)
+        per_config.append(run_fused_epilogue(sp, dev, flush, 10, hbm, tf_burst))
         resample = run_resample_chain(sp, dev, flush)
     if rank != 0:
         return

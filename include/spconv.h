@@ -262,6 +262,46 @@ SPCONV_API spconv_status_t spconv_subm_forward_algo(spconv_map_t map, spconv_dty
                                          spconv_algo_t algo, void* stream);
 
 /*
+ * Fused decoder epilogue of a forward (spconv_subm_forward_ex).  The
+ * pixal3d_mrp_mlx README ("Correction to the earlier scope") lists the ConvNeXt
+ * and ResBlock decoder blocks around the convolution; the lato.2_mrp_mlx README
+ * ("Status") lists the activations, norms and SparseResBlock of the shared core.
+ * The store of each output element then computes, in fp32,
+ *
+ *   y = act(conv + bias) (+ residual),  out = y rounded to the dtype,
+ *
+ * and, when `stats` is given, adds out and out^2 into per-channel sums over all
+ * rows (what a following LayerNorm / GroupNorm reads).
+ *
+ *   act       SPCONV_ACT_NONE, _RELU (max(y, 0)), _SILU (y / (1 + exp(-y))) or
+ *             _GELU (0.5 y (1 + erf(y / sqrt 2)), the exact form).
+ *   residual  device [n, cout] of the forward's dtype, 16-byte aligned, or NULL.
+ *             It may be `out` itself (each element is read before it is
+ *             written); it must not otherwise overlap out, and must not overlap x.
+ *   stats     device fp32 [2, cout], 16-byte aligned, or NULL: row 0 receives the
+ *             per-channel sum of the stored output, row 1 the sum of squares.  The
+ *             call zeroes it on `stream` first; the sums are accumulated with fp32
+ *             atomics, so their last bits depend on the order of the additions.
+ */
+typedef enum { SPCONV_ACT_NONE = 0, SPCONV_ACT_RELU = 1, SPCONV_ACT_SILU = 2, SPCONV_ACT_GELU = 3 } spconv_act_t;
+typedef struct {
+    spconv_act_t act;
+    const void* residual;
+    float* stats;
+} spconv_epilogue_t;
+
+/*
+ * spconv_subm_forward_algo with a fused epilogue.  `epi` may be NULL (no
+ * epilogue).  Same arguments, ownership, synchronisation (none) and errors as
+ * spconv_subm_forward_algo, plus SPCONV_ERR_INVALID_ARG for an unknown act, a
+ * misaligned residual or stats, or a residual overlapping x or partly overlapping
+ * out.  Both kernel families apply the epilogue.
+ */
+SPCONV_API spconv_status_t spconv_subm_forward_ex(spconv_map_t map, spconv_dtype_t dtype, const void* x, int32_t cin,
+                                                  const void* w, const void* bias, void* out, int32_t cout,
+                                                  const spconv_epilogue_t* epi, spconv_algo_t algo, void* stream);
+
+/*
  * Kernel families a forward can run on, for spconv_map_launch_counts.
  */
 typedef enum {

@@ -38,13 +38,20 @@ EXPORTED = ("spconv_build_map", "spconv_subm_forward", "spconv_free", "spconv_ma
             "spconv_debug_set_tile_rows", "spconv_build_neighbor_map_noalloc", "spconv_map_launch_counts",
             "spconv_map_stats", "spconv_debug_set_ring_depths", "spconv_build_map_ex", "spconv_downsample_build",
             "spconv_downsample_info", "spconv_downsample_amax", "spconv_upsample", "spconv_downsample_free",
-            "spconv_subdivide")
+            "spconv_subdivide", "spconv_subm_forward_ex")
 
 
 class _MapStats(ctypes.Structure):
     _fields_ = [("tiles", ctypes.c_int64), ("rows_per_tile", ctypes.c_int32), ("job_stride", ctypes.c_int32),
                 ("spans", ctypes.c_int64), ("span_cols", ctypes.c_int64), ("perm_dev", ctypes.c_void_p),
                 ("nbr_t_dev", ctypes.c_void_p), ("jobs_dev", ctypes.c_void_p), ("order_dev", ctypes.c_void_p)]
+
+
+class _Epilogue(ctypes.Structure):
+    _fields_ = [("act", ctypes.c_int), ("residual", ctypes.c_void_p), ("stats", ctypes.c_void_p)]
+
+
+ACTIVATIONS = {None: 0, "none": 0, "relu": 1, "silu": 2, "gelu": 3}
 
 
 class SpconvError(RuntimeError):
@@ -81,13 +88,15 @@ def _load() -> ctypes.CDLL:
     lib.spconv_upsample.argtypes = [vp, ctypes.c_int, vp, i32, vp, vp]
     lib.spconv_downsample_free.argtypes = [vp]
     lib.spconv_subdivide.argtypes = [vp, i64, vp, ctypes.c_int, vp, i32, vp, vp, vp]
+    lib.spconv_subm_forward_ex.argtypes = [vp, ctypes.c_int, vp, i32, vp, vp, vp, i32, ctypes.POINTER(_Epilogue),
+                                           ctypes.c_int, vp]
     lib.spconv_last_error.restype = ctypes.c_char_p
     for name in ("spconv_build_map", "spconv_subm_forward", "spconv_subm_forward_algo", "spconv_free",
                  "spconv_map_info", "spconv_map_check", "spconv_map_tile_rows", "spconv_debug_set_table_slots",
                  "spconv_debug_set_tile_rows", "spconv_build_neighbor_map_noalloc", "spconv_map_launch_counts",
                  "spconv_map_stats", "spconv_debug_set_ring_depths", "spconv_build_map_ex",
                  "spconv_downsample_build", "spconv_downsample_info", "spconv_downsample_amax", "spconv_upsample",
-                 "spconv_downsample_free", "spconv_subdivide"):
+                 "spconv_downsample_free", "spconv_subdivide", "spconv_subm_forward_ex"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -217,8 +226,12 @@ def spconv_build_map(coords: torch.Tensor, extent, kernel_size: int = 3, stream=
 
 
 def spconv_subm_forward(m: SubmMap, x: torch.Tensor, w: torch.Tensor, bias: torch.Tensor | None = None,
-                        out: torch.Tensor | None = None, algo: int = ALGO_AUTO, stream=None) -> torch.Tensor:
-    """One SubMConv3d layer: x [N, Cin], w [K^3, Cin, Cout], bias [Cout] -> out [N, Cout]."""
+                        out: torch.Tensor | None = None, algo: int = ALGO_AUTO, stream=None, act: str | None = None,
+                        residual: torch.Tensor | None = None, stats: torch.Tensor | None = None) -> torch.Tensor:
+    """One SubMConv3d layer: x [N, Cin], w [K^3, Cin, Cout], bias [Cout] -> out [N, Cout].
+    Fused epilogue (spconv_subm_forward_ex): out = act(conv + bias) (+ residual [N, Cout],
+    which may be ``out`` itself); ``stats``, a float32 CUDA tensor [2, Cout], receives the
+    per-channel sum and sum of squares of out."""
     _require()
     if x.dtype not in _DTYPES:
         raise ValueError("x must be float32 or bfloat16")
@@ -238,16 +251,33 @@ def spconv_subm_forward(m: SubmMap, x: torch.Tensor, w: torch.Tensor, bias: torc
     # tensor, or one on another GPU than the map, must never reach it.
     if not x.is_cuda or x.device != m.device or (out is not None and out.device != x.device):
         raise ValueError(f"x, w, bias and out must be CUDA tensors on the map's device {m.device}")
+    if act not in ACTIVATIONS:
+        raise ValueError(f"act must be one of {sorted(k for k in ACTIVATIONS if k)} or None")
+    if residual is not None and (residual.shape != (m.n, cout) or residual.dtype != x.dtype
+                                 or residual.device != x.device or not residual.is_contiguous()):
+        raise ValueError("residual must be a contiguous [N, Cout] tensor of x's dtype on x's device")
+    if stats is not None and (stats.shape != (2, cout) or stats.dtype != torch.float32
+                              or stats.device != x.device or not stats.is_contiguous()):
+        raise ValueError("stats must be a contiguous float32 [2, Cout] tensor on x's device")
     x, w = x.contiguous(), w.contiguous()
     bias = None if bias is None else bias.contiguous()
     if out is None:
         out = torch.empty((m.n, cout), dtype=x.dtype, device=x.device)
     if m.n == 0:
+        if stats is not None:
+            stats.zero_()
         return out
     with torch.cuda.device(x.device):
-        _check(lib.spconv_subm_forward_algo(m.handle, _DTYPES[x.dtype], x.data_ptr(), cin, w.data_ptr(),
-                                            None if bias is None else bias.data_ptr(), out.data_ptr(), cout,
-                                            algo, _stream(stream)))
+        if ACTIVATIONS[act] or residual is not None or stats is not None:
+            epi = _Epilogue(ACTIVATIONS[act], None if residual is None else residual.data_ptr(),
+                            None if stats is None else stats.data_ptr())
+            _check(lib.spconv_subm_forward_ex(m.handle, _DTYPES[x.dtype], x.data_ptr(), cin, w.data_ptr(),
+                                              None if bias is None else bias.data_ptr(), out.data_ptr(), cout,
+                                              ctypes.byref(epi), algo, _stream(stream)))
+        else:
+            _check(lib.spconv_subm_forward_algo(m.handle, _DTYPES[x.dtype], x.data_ptr(), cin, w.data_ptr(),
+                                                None if bias is None else bias.data_ptr(), out.data_ptr(), cout,
+                                                algo, _stream(stream)))
     return out
 
 
@@ -415,6 +445,6 @@ __all__ = ["OK", "INVALID_ARG", "UNSUPPORTED", "COORD_RANGE", "DUPLICATE", "TABL
            "spconv_debug_set_table_slots", "spconv_debug_set_tile_rows", "spconv_debug_set_ring_depths",
            "spconv_build_neighbor_map_noalloc", "lib", "Downsample", "spconv_downsample_build",
            "spconv_downsample_amax", "spconv_upsample", "spconv_subdivide", "MAP_DEFAULT", "MAP_FLIP_KERNEL",
-           "MAP_SORTED_KEYS",
+           "MAP_SORTED_KEYS", "MAP_HASH_TABLE", "ACTIVATIONS",
            "LIB_PATH", "EXPORTED",
            "ALGO_AUTO", "ALGO_SIMT", "ALGO_TCGEN05", "KERNEL_SIMT", "KERNEL_TCGEN05", "KERNEL_NAMES"]

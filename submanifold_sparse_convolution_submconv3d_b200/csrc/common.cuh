@@ -82,6 +82,22 @@ inline int choose_win_rows(int64_t n, int num_sms) {
     return best;
 }
 
+// Fused epilogue of a forward: y = act(conv + bias) (+ residual), stored; per
+// channel sums of the stored value and its square into stats[0..cout) and
+// stats[cout..2 cout) when stats is set.
+struct Epilogue {
+    int act = SPCONV_ACT_NONE;
+    const void* residual = nullptr;
+    float* stats = nullptr;
+};
+
+__device__ __forceinline__ float epi_act(int act, float y) {
+    if (act == SPCONV_ACT_RELU) return fmaxf(y, 0.0f);
+    if (act == SPCONV_ACT_SILU) return y / (1.0f + expf(-y));
+    if (act == SPCONV_ACT_GELU) return 0.5f * y * (1.0f + erff(y * 0.70710678118654752f));
+    return y;
+}
+
 // The map handle (defined here so the launchers can read it).
 struct MapData {
     int64_t n = 0;
@@ -163,7 +179,7 @@ cudaError_t launch_win_meta(const int32_t* nbr, const int32_t* sorted_rows, int6
 cudaError_t launch_win_cost(const uint32_t* jobs, int64_t tiles, uint32_t* keys, cudaStream_t stream);
 
 cudaError_t launch_forward_simt(const MapData& m, spconv_dtype_t dtype, const void* x, int cin, const void* w,
-                                const void* bias, void* out, int cout, cudaStream_t stream);
+                                const void* bias, void* out, int cout, const Epilogue& epi, cudaStream_t stream);
 
 // Test hook of the tensor-core forward: force the weight-ring slots and B-ring
 // units of later launches (0, 0: automatic).
@@ -171,7 +187,7 @@ void set_forced_ring_depths(int sa, int ub);
 
 // Returns SPCONV_OK, SPCONV_ERR_UNSUPPORTED (shape not handled) or SPCONV_ERR_CUDA.
 spconv_status_t launch_forward_tcgen05(const MapData& m, const void* x, int cin, const void* w,
-                                       const void* bias, void* out, int cout, cudaStream_t stream,
-                                       cudaError_t* cuda_err);
+                                       const void* bias, void* out, int cout, const Epilogue& epi,
+                                       cudaStream_t stream, cudaError_t* cuda_err);
 
 }  // namespace spconv

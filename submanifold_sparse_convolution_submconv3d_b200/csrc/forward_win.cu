@@ -144,6 +144,9 @@ struct WinParams {
     const __nv_bfloat16* bias;
     __nv_bfloat16* out;
     int cout;
+    int act;                           // fused epilogue: spconv_act_t of conv + bias
+    const __nv_bfloat16* residual;     // [n, cout] added after the activation, or null (may equal out)
+    float* stats;                      // [2, cout] per-channel sum and sum of squares of out, or null
     unsigned int* err;
     int sa, ub;                 // weight-ring slots, B-ring units
     int idx_buf_elems;          // int32 entries of one tile index buffer
@@ -210,7 +213,7 @@ __device__ __forceinline__ const uint32_t* slot_rec(const uint8_t* slot) {
     return reinterpret_cast<const uint32_t*>(slot + 16);
 }
 
-template <int BM, int KC>
+template <int BM, int KC, bool kFused>
 __global__ void __launch_bounds__(kThreads, 1)
     k_subm_win(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap, const WinParams p) {
     using L = WinLayout<BM, KC>;
@@ -700,6 +703,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
+            float s1 = 0.0f, s2 = 0.0f;  // this lane's channel statistics over the tile (fused epilogue)
 #pragma unroll
             for (int c4 = 0; c4 < kChunksPerWarp; ++c4) {
                 const int cc = half + kEpiGroups * c4;
@@ -709,10 +713,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_wait_ld();
 #pragma unroll
                     for (int hp = 0; hp < 32 / L::kStageRows; ++hp) {
-                        if (lane_ok) {
+                        if constexpr (!kFused) {
+                            if (lane_ok) {
+#pragma unroll
+                                for (int e = 0; e < L::kStageRows; ++e)
+                                    stg[e * L::kChPerWarp + lane] =
+                                        __float2bfloat16_rn(v[hp * L::kStageRows + e] + bv);
+                            }
+                        } else {
+                            // fused epilogue: act(conv + bias) (+ residual) in fp32, then the
+                            // rounded value is stored and counted in the statistics
+                            int ro[L::kStageRows];  // output rows of these columns (-1: none)
 #pragma unroll
                             for (int e = 0; e < L::kStageRows; ++e)
-                                stg[e * L::kChPerWarp + lane] = __float2bfloat16_rn(v[hp * L::kStageRows + e] + bv);
+                                ro[e] = __shfl_sync(0xffffffffu, orow[c4], hp * L::kStageRows + e);
+                            if (lane_ok) {
+#pragma unroll
+                                for (int e = 0; e < L::kStageRows; ++e) {
+                                    float y = epi_act(p.act, v[hp * L::kStageRows + e] + bv);
+                                    if (p.residual && ro[e] >= 0)
+                                        y += __bfloat162float(p.residual[(int64_t)ro[e] * p.cout + ch_base + lane]);
+                                    const __nv_bfloat16 q = __float2bfloat16_rn(y);
+                                    stg[e * L::kChPerWarp + lane] = q;
+                                    if (ro[e] >= 0) {
+                                        const float f = __bfloat162float(q);
+                                        s1 += f;
+                                        s2 += f * f;
+                                    }
+                                }
+                            }
                         }
                         __syncwarp();
 #pragma unroll
@@ -726,6 +755,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         __syncwarp();
                     }
+                }
+            }
+            if constexpr (kFused) {
+                if (p.stats && lane_ok) {
+                    atomicAdd(p.stats + ch_base + lane, s1);
+                    atomicAdd(p.stats + p.cout + ch_base + lane, s2);
                 }
             }
             tc_fence_before();
@@ -791,7 +826,7 @@ bool choose_depths(int rows, int max_cols, int* sa, int* ub) {
 
 template <int BM, int KC>
 spconv_status_t launch(const MapData& m, const void* x, int cin, const void* w, const void* bias, void* out,
-                       int cout, cudaStream_t stream, cudaError_t* ce) {
+                       int cout, const Epilogue& epi, cudaStream_t stream, cudaError_t* ce) {
     using L = WinLayout<BM, KC>;
     EncodeTiledFn enc = encode_fn();
     if (!enc) {
@@ -845,19 +880,23 @@ spconv_status_t launch(const MapData& m, const void* x, int cin, const void* w, 
         *ce = de;
         return SPCONV_ERR_CUDA;
     }
+    // the fused-epilogue instantiation runs only when an epilogue op is asked for,
+    // so plain layers keep the plain store
+    const bool fused = epi.act != SPCONV_ACT_NONE || epi.residual != nullptr || epi.stats != nullptr;
+    auto kernel = fused ? k_subm_win<BM, KC, true> : k_subm_win<BM, KC, false>;
     {   // the shared-memory opt-in is per device context and instantiation
         static std::mutex attr_mu;
-        static std::vector<char> attr_done;
+        static std::vector<char> attr_done;  // bit 0: plain, bit 1: fused
         std::lock_guard<std::mutex> lock(attr_mu);
         if (dev >= (int)attr_done.size()) attr_done.resize((size_t)dev + 1, 0);
-        if (!attr_done[dev]) {
-            const cudaError_t ae =
-                cudaFuncSetAttribute(k_subm_win<BM, KC>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+        const char bit = fused ? 2 : 1;
+        if (!(attr_done[dev] & bit)) {
+            const cudaError_t ae = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
             if (ae != cudaSuccess) {
                 *ce = ae;
                 return SPCONV_ERR_CUDA;
             }
-            attr_done[dev] = 1;
+            attr_done[dev] |= bit;
         }
     }
     // this launch's work counter: one of the map's slots in turn (zeroed by the
@@ -884,9 +923,12 @@ spconv_status_t launch(const MapData& m, const void* x, int cin, const void* w, 
     p.ub = ub;
     p.idx_buf_elems = L::idx_buf_bytes(max_cols) / 4;
     p.rows_tma = rows_tma ? 1 : 0;
+    p.act = epi.act;
+    p.residual = static_cast<const __nv_bfloat16*>(epi.residual);
+    p.stats = epi.stats;
     const int64_t units = m.win_tiles * p.cblocks;
     const int64_t grid = units < m.num_sms ? units : m.num_sms;
-    k_subm_win<BM, KC><<<(unsigned)grid, kThreads, smem, stream>>>(map, xmap, p);
+    kernel<<<(unsigned)grid, kThreads, smem, stream>>>(map, xmap, p);
     *ce = cudaGetLastError();
     return *ce == cudaSuccess ? SPCONV_OK : SPCONV_ERR_CUDA;
 }
@@ -899,22 +941,23 @@ void set_forced_ring_depths(int sa, int ub) {
 }
 
 spconv_status_t launch_forward_tcgen05(const MapData& m, const void* x, int cin, const void* w, const void* bias,
-                                       void* out, int cout, cudaStream_t stream, cudaError_t* ce) {
+                                       void* out, int cout, const Epilogue& epi, cudaStream_t stream,
+                                       cudaError_t* ce) {
     *ce = cudaSuccess;
     if (cin % 16 != 0 || cout % 64 != 0) return SPCONV_ERR_UNSUPPORTED;
     if (m.n == 0) return SPCONV_OK;
     const bool bm128 = cout % 128 == 0;
     const int kc = cin % 128 == 0 ? 128 : (cin % 64 == 0 ? 64 : (cin % 32 == 0 ? 32 : 16));
     if (bm128) {
-        if (kc == 128) return launch<128, 128>(m, x, cin, w, bias, out, cout, stream, ce);
-        if (kc == 64) return launch<128, 64>(m, x, cin, w, bias, out, cout, stream, ce);
-        if (kc == 32) return launch<128, 32>(m, x, cin, w, bias, out, cout, stream, ce);
-        return launch<128, 16>(m, x, cin, w, bias, out, cout, stream, ce);
+        if (kc == 128) return launch<128, 128>(m, x, cin, w, bias, out, cout, epi, stream, ce);
+        if (kc == 64) return launch<128, 64>(m, x, cin, w, bias, out, cout, epi, stream, ce);
+        if (kc == 32) return launch<128, 32>(m, x, cin, w, bias, out, cout, epi, stream, ce);
+        return launch<128, 16>(m, x, cin, w, bias, out, cout, epi, stream, ce);
     }
-    if (kc == 128) return launch<64, 128>(m, x, cin, w, bias, out, cout, stream, ce);
-    if (kc == 64) return launch<64, 64>(m, x, cin, w, bias, out, cout, stream, ce);
-    if (kc == 32) return launch<64, 32>(m, x, cin, w, bias, out, cout, stream, ce);
-    return launch<64, 16>(m, x, cin, w, bias, out, cout, stream, ce);
+    if (kc == 128) return launch<64, 128>(m, x, cin, w, bias, out, cout, epi, stream, ce);
+    if (kc == 64) return launch<64, 64>(m, x, cin, w, bias, out, cout, epi, stream, ce);
+    if (kc == 32) return launch<64, 32>(m, x, cin, w, bias, out, cout, epi, stream, ce);
+    return launch<64, 16>(m, x, cin, w, bias, out, cout, epi, stream, ce);
 }
 
 }  // namespace spconv

@@ -330,9 +330,9 @@ spconv_status_t spconv_map_check(spconv_map_t map, void* stream_) {
     return SPCONV_OK;
 }
 
-spconv_status_t spconv_subm_forward_algo(spconv_map_t map, spconv_dtype_t dtype, const void* x, int32_t cin,
-                                         const void* w, const void* bias, void* out, int32_t cout,
-                                         spconv_algo_t algo, void* stream_) {
+spconv_status_t spconv_subm_forward_ex(spconv_map_t map, spconv_dtype_t dtype, const void* x, int32_t cin,
+                                       const void* w, const void* bias, void* out, int32_t cout,
+                                       const spconv_epilogue_t* epi_, spconv_algo_t algo, void* stream_) {
     g_last_error.clear();
     if (!map) return fail(SPCONV_ERR_INVALID_ARG, "null map");
     if (dtype != SPCONV_F32 && dtype != SPCONV_BF16) return fail(SPCONV_ERR_INVALID_ARG, "dtype must be SPCONV_F32 or SPCONV_BF16");
@@ -359,7 +359,30 @@ spconv_status_t spconv_subm_forward_algo(spconv_map_t map, spconv_dtype_t dtype,
         const size_t xbytes = (size_t)map->d.n * cin * esz, obytes = (size_t)map->d.n * cout * esz;
         if (ob < xb + xbytes && xb < ob + obytes) return fail(SPCONV_ERR_INVALID_ARG, "out overlaps x");
     }
+    spconv::Epilogue epi;
+    if (epi_) {
+        if (epi_->act < SPCONV_ACT_NONE || epi_->act > SPCONV_ACT_GELU)
+            return fail(SPCONV_ERR_INVALID_ARG, "unknown activation");
+        epi.act = epi_->act;
+        epi.residual = epi_->residual;
+        epi.stats = epi_->stats;
+        if (epi.residual) {
+            if (!aligned16(epi.residual)) return fail(SPCONV_ERR_INVALID_ARG, "residual must be 16-byte aligned");
+            const char* rb = static_cast<const char*>(epi.residual);
+            const char* xb = static_cast<const char*>(x);
+            const char* ob = static_cast<const char*>(out);
+            const size_t rbytes = (size_t)map->d.n * cout * esz, xbytes = (size_t)map->d.n * cin * esz;
+            if (rb < xb + xbytes && xb < rb + rbytes) return fail(SPCONV_ERR_INVALID_ARG, "residual overlaps x");
+            if (rb != ob && rb < ob + rbytes && ob < rb + rbytes)
+                return fail(SPCONV_ERR_INVALID_ARG, "residual partly overlaps out");
+        }
+        if (epi.stats && !aligned16(epi.stats)) return fail(SPCONV_ERR_INVALID_ARG, "stats must be 16-byte aligned");
+    }
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    if (epi.stats) {
+        const cudaError_t me = cudaMemsetAsync(epi.stats, 0, (size_t)2 * cout * sizeof(float), stream);
+        if (me != cudaSuccess) return fail_cuda(me, "zeroing stats");
+    }
     if (algo == SPCONV_ALGO_TCGEN05 && dtype != SPCONV_BF16)
         return fail(SPCONV_ERR_UNSUPPORTED, "the tcgen05 kernel is bf16 only");
     // AUTO: bf16 with cout % 64 == 0 runs on the tensor cores; fp32 and other bf16
@@ -368,22 +391,28 @@ spconv_status_t spconv_subm_forward_algo(spconv_map_t map, spconv_dtype_t dtype,
     const bool tc_shape = dtype == SPCONV_BF16 && cout % 64 == 0;
     if (algo == SPCONV_ALGO_TCGEN05 || (algo == SPCONV_ALGO_AUTO && tc_shape)) {
         cudaError_t ce = cudaSuccess;
-        const spconv_status_t s = spconv::launch_forward_tcgen05(map->d, x, cin, w, bias, out, cout, stream, &ce);
+        const spconv_status_t s = spconv::launch_forward_tcgen05(map->d, x, cin, w, bias, out, cout, epi, stream, &ce);
         if (s == SPCONV_ERR_CUDA) return fail_cuda(ce, "tcgen05 forward");
         if (s != SPCONV_OK)
             return fail(s, "the tcgen05 kernel does not take this shape (bf16 with cout % 64 == 0 and cin % 16 == 0)");
         map->launches[SPCONV_KERNEL_TCGEN05].fetch_add(1);
         return SPCONV_OK;
     }
-    cudaError_t e = spconv::launch_forward_simt(map->d, dtype, x, cin, w, bias, out, cout, stream);
+    cudaError_t e = spconv::launch_forward_simt(map->d, dtype, x, cin, w, bias, out, cout, epi, stream);
     if (e != cudaSuccess) return fail_cuda(e, "simt forward");
     map->launches[SPCONV_KERNEL_SIMT].fetch_add(1);
     return SPCONV_OK;
 }
 
+spconv_status_t spconv_subm_forward_algo(spconv_map_t map, spconv_dtype_t dtype, const void* x, int32_t cin,
+                                         const void* w, const void* bias, void* out, int32_t cout,
+                                         spconv_algo_t algo, void* stream) {
+    return spconv_subm_forward_ex(map, dtype, x, cin, w, bias, out, cout, nullptr, algo, stream);
+}
+
 spconv_status_t spconv_subm_forward(spconv_map_t map, spconv_dtype_t dtype, const void* x, int32_t cin,
                                     const void* w, const void* bias, void* out, int32_t cout, void* stream) {
-    return spconv_subm_forward_algo(map, dtype, x, cin, w, bias, out, cout, SPCONV_ALGO_AUTO, stream);
+    return spconv_subm_forward_ex(map, dtype, x, cin, w, bias, out, cout, nullptr, SPCONV_ALGO_AUTO, stream);
 }
 
 spconv_status_t spconv_map_launch_counts(spconv_map_t map, int64_t* counts, int32_t ncounts) {
