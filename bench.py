@@ -58,12 +58,13 @@ CONFIG = {
     "grid": 128, "voxels": 209715, "cin": 128, "cout": 128, "kernel_size": 3, "layers_per_step": LAYERS,
     "l2": "flushed before every timed step (512 MB write)",
     "launch": "each step is one captured CUDA graph of the ten layers",
+    "map": "built with SPCONV_MAP_SHORT_TILES (128-row tiles: the layers take 128 input channels)",
 }
-PER_CONFIG = (  # (workload, layer index, label)
-    ("shells", 0, "shells k=3 64->64"),
-    ("batched", 0, "batched k=3 512->512"),
-    ("batched", 1, "batched k=1 512->512"),
-    ("large", 0, "large k=3 32->64"),
+PER_CONFIG = (  # (workload, layer index, label, short tiles: the layer takes >= 128 input channels)
+    ("shells", 0, "shells k=3 64->64", False),
+    ("batched", 0, "batched k=3 512->512", True),
+    ("batched", 1, "batched k=1 512->512", True),
+    ("large", 0, "large k=3 32->64", False),
 )
 
 # DRAM traffic of one forward launch from a committed ncu capture
@@ -272,13 +273,13 @@ def run_per_config(sp, dev, flush, reps: int, hbm: float, tflops: float, cpu: bo
     import torch
     results = []
     cache = {}
-    for name, li, label in PER_CONFIG:
+    for name, li, label, short in PER_CONFIG:
         wl = cache.setdefault(name, workloads.make_workload(name, 0))
         layer = wl.layers[li]
         ks = layer.kernel_size
         kvol, cin, cout = layer.w.shape
         coords_d = torch.from_numpy(wl.coords).to(dev)
-        m = sp.spconv_build_map(coords_d, wl.grid, ks)
+        m = sp.spconv_build_map(coords_d, wl.grid, ks, short_tiles=short)
         x = torch.from_numpy(wl.x).to(dev, torch.bfloat16)
         w = torch.from_numpy(layer.w).to(dev, torch.bfloat16)
         b = torch.from_numpy(layer.bias).to(dev, torch.bfloat16)
@@ -340,7 +341,7 @@ def run_fused_epilogue(sp, dev, flush, reps: int, hbm: float, tflops: float) -> 
     import torch
     wl = workloads.make_workload(WORKLOAD, 0, n_layers=1)
     layer = wl.layers[0]
-    m = sp.spconv_build_map(torch.from_numpy(wl.coords).to(dev), wl.grid, 3)
+    m = sp.spconv_build_map(torch.from_numpy(wl.coords).to(dev), wl.grid, 3, short_tiles=True)
     x = torch.from_numpy(wl.x).to(dev, torch.bfloat16)
     w = torch.from_numpy(layer.w).to(dev, torch.bfloat16)
     b = torch.from_numpy(layer.bias).to(dev, torch.bfloat16)
@@ -526,7 +527,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     x0 = bufs[0].clone()
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
 
-    m = sp.spconv_build_map(coords_d, wl.grid, 3)
+    m = sp.spconv_build_map(coords_d, wl.grid, 3, short_tiles=True)
     pairs = m.pairs
     st = m.stats()
 
@@ -565,7 +566,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         flush.fill_(1.0)
         torch.cuda.synchronize()
         t0 = time.perf_counter()
-        mm = sp.spconv_build_map(coords_d, wl.grid, 3)
+        mm = sp.spconv_build_map(coords_d, wl.grid, 3, short_tiles=True)
         build_ms.append((time.perf_counter() - t0) * 1e3)
         mm.free()
 
@@ -581,7 +582,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         xa = x_h.to(dev, non_blocking=True)
         wd = [w.to(dev, non_blocking=True) for w in w_h]
         bd = [b.to(dev, non_blocking=True) for b in b_h]
-        me = sp.spconv_build_map(c_d, wl.grid, 3)
+        me = sp.spconv_build_map(c_d, wl.grid, 3, short_tiles=True)
         xb = torch.empty_like(xa)
         pp = [xa, xb]
         for li in range(LAYERS):

@@ -120,6 +120,10 @@ SPCONV_API spconv_status_t spconv_build_map(const int32_t* coords, int64_t n, co
  *                           (SPCONV_ERR_UNSUPPORTED otherwise); never reports
  *                           SPCONV_ERR_TABLE_FULL.
  *   SPCONV_MAP_HASH_TABLE   build with the hash table whatever the size.
+ *   SPCONV_MAP_SHORT_TILES  cut the sorted rows into 128-row tiles instead of 192:
+ *                           faster for layers with 128 or more input channels
+ *                           (their 16 KB gather units leave room for fewer jobs
+ *                           in flight), slower for narrower ones.  Same results.
  * With neither dictionary flag the library picks one: the hash table below
  * 2^20 voxels, the sorted keys from 2^20 voxels on when the key bits fit (and
  * the hash table whenever spconv_debug_set_table_slots forces a table size).
@@ -129,7 +133,8 @@ typedef enum {
     SPCONV_MAP_DEFAULT = 0,
     SPCONV_MAP_FLIP_KERNEL = 1,
     SPCONV_MAP_SORTED_KEYS = 2,
-    SPCONV_MAP_HASH_TABLE = 4
+    SPCONV_MAP_HASH_TABLE = 4,
+    SPCONV_MAP_SHORT_TILES = 8
 } spconv_map_flags_t;
 
 /*
@@ -189,9 +194,9 @@ SPCONV_API spconv_status_t spconv_map_info(spconv_map_t map, int64_t* n, int32_t
 
 /*
  * Rows per tile (a multiple of 16, at most 256) that the tensor-core forward uses
- * with this map: chosen at build time to even out the rows of the busiest SM when
- * the tiles are dealt out over the device's SMs, or forced by
- * spconv_debug_set_tile_rows.  For reports and tests; no device work.
+ * with this map: 192, or 128 with SPCONV_MAP_SHORT_TILES; a set too small to give
+ * every SM a 192-row tile takes the height in [128, 192] that evens out the rows
+ * of the busiest SM; spconv_debug_set_tile_rows forces it.  For reports and tests; no device work.
  * A null `map` or `rows` returns SPCONV_ERR_INVALID_ARG.
  */
 SPCONV_API spconv_status_t spconv_map_tile_rows(spconv_map_t map, int32_t* rows);

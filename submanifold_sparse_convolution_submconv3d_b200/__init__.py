@@ -26,7 +26,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libspconv_b200.so")
 
 OK, INVALID_ARG, UNSUPPORTED, COORD_RANGE, DUPLICATE, TABLE_FULL, OOM, CUDA_ERROR, TIMEOUT = range(9)
-MAP_DEFAULT, MAP_FLIP_KERNEL, MAP_SORTED_KEYS, MAP_HASH_TABLE = 0, 1, 2, 4
+MAP_DEFAULT, MAP_FLIP_KERNEL, MAP_SORTED_KEYS, MAP_HASH_TABLE, MAP_SHORT_TILES = 0, 1, 2, 4, 8
 ALGO_AUTO, ALGO_SIMT, ALGO_TCGEN05 = 0, 1, 2
 KERNEL_SIMT, KERNEL_TCGEN05 = 0, 1
 KERNEL_NAMES = ("simt", "tcgen05")
@@ -204,15 +204,17 @@ def _coords_arg(coords: torch.Tensor) -> torch.Tensor:
 
 
 def spconv_build_map(coords: torch.Tensor, extent, kernel_size: int = 3, stream=None, flip_kernel: bool = False,
-                     sorted_keys: bool | None = None) -> SubmMap:
+                     sorted_keys: bool | None = None, short_tiles: bool = False) -> SubmMap:
     """Build the neighbour map of int32 [N, 4] (b, x, y, z) CUDA coordinates.
     ``flip_kernel`` gathers p - d_k; ``sorted_keys`` True / False forces the sorted-key
-    or the hash-table dictionary (same map); None lets the library choose by size."""
+    or the hash-table dictionary (same map); None lets the library choose by size;
+    ``short_tiles`` cuts the forward's tiles at 128 rows (faster for layers with 128
+    or more input channels)."""
     _require()
     coords = _coords_arg(coords)
     ext = (ctypes.c_int32 * 3)(*[int(v) for v in extent])
     handle = ctypes.c_void_p()
-    flags = (MAP_FLIP_KERNEL if flip_kernel else 0) | \
+    flags = (MAP_FLIP_KERNEL if flip_kernel else 0) | (MAP_SHORT_TILES if short_tiles else 0) | \
         {None: 0, True: MAP_SORTED_KEYS, False: MAP_HASH_TABLE}[sorted_keys]
     with torch.cuda.device(coords.device):
         ptr = coords.data_ptr() if coords.numel() else None
@@ -445,6 +447,6 @@ __all__ = ["OK", "INVALID_ARG", "UNSUPPORTED", "COORD_RANGE", "DUPLICATE", "TABL
            "spconv_debug_set_table_slots", "spconv_debug_set_tile_rows", "spconv_debug_set_ring_depths",
            "spconv_build_neighbor_map_noalloc", "lib", "Downsample", "spconv_downsample_build",
            "spconv_downsample_amax", "spconv_upsample", "spconv_subdivide", "MAP_DEFAULT", "MAP_FLIP_KERNEL",
-           "MAP_SORTED_KEYS", "MAP_HASH_TABLE", "ACTIVATIONS",
+           "MAP_SORTED_KEYS", "MAP_HASH_TABLE", "MAP_SHORT_TILES", "ACTIVATIONS",
            "LIB_PATH", "EXPORTED",
            "ALGO_AUTO", "ALGO_SIMT", "ALGO_TCGEN05", "KERNEL_SIMT", "KERNEL_TCGEN05", "KERNEL_NAMES"]

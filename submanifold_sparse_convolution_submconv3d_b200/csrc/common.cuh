@@ -64,14 +64,21 @@ __host__ __device__ inline int win_job_k(uint32_t j) { return (int)(j & 31u); }
 __host__ __device__ inline int win_job_w0(uint32_t j) { return (int)((j >> 8) & 31u); }
 __host__ __device__ inline int win_job_nw(uint32_t j) { return (int)((j >> 16) & 31u); }
 
-// Window-tile height for n rows on num_sms SMs: the multiple of kWinCols in
-// [128, kWinMaxRows] that minimises the rows of the busiest SM when tiles are
-// dealt out round-robin (ties: the taller tile).
-inline int choose_win_rows(int64_t n, int num_sms) {
-    if (n <= 0 || num_sms <= 0) return kWinMaxRows;
-    int best = kWinMaxRows;
+// Window-tile height for n rows on num_sms SMs.  Measured on B200 (128^3 random,
+// 256^3 and 512^3 shells, 4 x 64^3 shells; 64-256-row tiles): 192 rows is the
+// fastest height for 32- and 64-channel chunks, 128 rows for 128-channel chunks,
+// whose 16 KB gather units make the B ring shallow (so the short-tiles option,
+// for maps whose layers take 128 or more input channels, picks 128).  A set too
+// small to give every SM a 192-row tile takes the multiple of kWinCols in
+// [128, 192] that minimises the rows of the busiest SM (ties: the taller tile).
+constexpr int kTileRowsDefault = 192;
+constexpr int kTileRowsShort = 128;
+inline int choose_win_rows(int64_t n, int num_sms, bool short_tiles) {
+    if (short_tiles) return kTileRowsShort;
+    if (n <= 0 || num_sms <= 0 || n >= (int64_t)num_sms * kTileRowsDefault) return kTileRowsDefault;
+    int best = kTileRowsDefault;
     int64_t best_load = -1;
-    for (int r = kWinMaxRows; r >= 128; r -= kWinCols) {
+    for (int r = kTileRowsDefault; r >= kTileRowsShort; r -= kWinCols) {
         const int64_t tiles = (n + r - 1) / r;
         const int64_t load = (tiles + num_sms - 1) / num_sms * r;
         if (best_load < 0 || load < best_load) {

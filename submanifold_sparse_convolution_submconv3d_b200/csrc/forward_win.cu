@@ -72,6 +72,10 @@ constexpr int kThreads = 32 * (kWarpPrep + 1);          // 480
 constexpr int kCmdSlots = 16;
 constexpr uint32_t kCmdRelA = 1, kCmdInit = 2, kCmdFirst = 4, kCmdTileEnd = 8, kCmdExit = 16;
 constexpr int kEpiGroups = kEpiWarps / 4;  // epilogue warps per TMEM lane quarter
+// Kernel instantiations by epilogue: the plain store, and the fused epilogue with
+// ReLU or none (chosen at run time), SiLU or GELU, so no instantiation carries the
+// code of the activations it does not run.
+constexpr int kEpiPlain = 0, kEpiRelu = 1, kEpiSilu = 2, kEpiGelu = 3;
 static_assert(kEpiWarps % 4 == 0 && kWinMaxRows / 32 % kEpiGroups == 0, "whole lane quarters, whole chunks");
 constexpr int kAccBufs = 2;
 constexpr int kIdxBufs = 2;
@@ -213,7 +217,7 @@ __device__ __forceinline__ const uint32_t* slot_rec(const uint8_t* slot) {
     return reinterpret_cast<const uint32_t*>(slot + 16);
 }
 
-template <int BM, int KC, bool kFused>
+template <int BM, int KC, int kEpi>
 __global__ void __launch_bounds__(kThreads, 1)
     k_subm_win(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap, const WinParams p) {
     using L = WinLayout<BM, KC>;
@@ -698,6 +702,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 orow[c4] = col < t_eff ? (p.perm ? p.perm[row_t0 + col] : (int)(row_t0 + col)) : -1;
             }
             const float bv = (p.bias && lane_ok) ? __bfloat162float(p.bias[ch_base + lane]) : 0.0f;
+            if constexpr (kEpi != kEpiPlain) {
+                // the residual slices of this warp's rows into L2 while the MMAs run
+                if (p.residual) {
+#pragma unroll
+                    for (int c4 = 0; c4 < kChunksPerWarp; ++c4)
+                        if (orow[c4] >= 0) prefetch_l2(p.residual + (int64_t)orow[c4] * p.cout + ch_base);
+                }
+            }
             if (!warp_wait_bar<kSleepEpilogue>(accF0 + 8 * buf, (uint32_t)(i >> 1) & 1u, abort_flag, p.err)) {
                 aborted = true;
                 break;
@@ -713,7 +725,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_wait_ld();
 #pragma unroll
                     for (int hp = 0; hp < 32 / L::kStageRows; ++hp) {
-                        if constexpr (!kFused) {
+                        if constexpr (kEpi == kEpiPlain) {
                             if (lane_ok) {
 #pragma unroll
                                 for (int e = 0; e < L::kStageRows; ++e)
@@ -723,19 +735,40 @@ __global__ void __launch_bounds__(kThreads, 1)
                         } else {
                             // fused epilogue: act(conv + bias) (+ residual) in fp32, then the
                             // rounded value is stored and counted in the statistics
-                            int ro[L::kStageRows];  // output rows of these columns (-1: none)
+                            const int col0 = cc * 32 + hp * L::kStageRows;  // tile column of row e = col0 + e
+                            float rv[L::kStageRows];  // residual elements (0 when there is none)
+                            if (p.residual) {
+                                // the output rows of these columns, then their residual
+                                // elements, loaded together (a missing row reads row 0)
+                                int ro[L::kStageRows];
 #pragma unroll
-                            for (int e = 0; e < L::kStageRows; ++e)
-                                ro[e] = __shfl_sync(0xffffffffu, orow[c4], hp * L::kStageRows + e);
+                                for (int e = 0; e < L::kStageRows; ++e)
+                                    ro[e] = __shfl_sync(0xffffffffu, orow[c4], hp * L::kStageRows + e);
+#pragma unroll
+                                for (int e = 0; e < L::kStageRows; ++e)
+                                    rv[e] = lane_ok ? __bfloat162float(p.residual[(int64_t)(ro[e] > 0 ? ro[e] : 0) *
+                                                                                      p.cout + ch_base + lane])
+                                                    : 0.0f;
+                            } else {
+#pragma unroll
+                                for (int e = 0; e < L::kStageRows; ++e) rv[e] = 0.0f;
+                            }
                             if (lane_ok) {
 #pragma unroll
                                 for (int e = 0; e < L::kStageRows; ++e) {
-                                    float y = epi_act(p.act, v[hp * L::kStageRows + e] + bv);
-                                    if (p.residual && ro[e] >= 0)
-                                        y += __bfloat162float(p.residual[(int64_t)ro[e] * p.cout + ch_base + lane]);
-                                    const __nv_bfloat16 q = __float2bfloat16_rn(y);
+                                    float y = v[hp * L::kStageRows + e] + bv;
+                                    if constexpr (kEpi == kEpiRelu) {
+                                        if (p.act == SPCONV_ACT_RELU) y = fmaxf(y, 0.0f);
+                                    } else if constexpr (kEpi == kEpiSilu) {
+                                        // fast exponential and division: their error is far below the
+                                        // bf16 rounding of out (a huge denominator gives -0 for y << 0)
+                                        y = __fdividef(y, 1.0f + __expf(-y));
+                                    } else {
+                                        y = epi_act(SPCONV_ACT_GELU, y);
+                                    }
+                                    const __nv_bfloat16 q = __float2bfloat16_rn(y + rv[e]);
                                     stg[e * L::kChPerWarp + lane] = q;
-                                    if (ro[e] >= 0) {
+                                    if (col0 + e < t_eff) {
                                         const float f = __bfloat162float(q);
                                         s1 += f;
                                         s2 += f * f;
@@ -757,7 +790,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            if constexpr (kFused) {
+            if constexpr (kEpi != kEpiPlain) {
                 if (p.stats && lane_ok) {
                     atomicAdd(p.stats + ch_base + lane, s1);
                     atomicAdd(p.stats + p.cout + ch_base + lane, s2);
@@ -883,13 +916,18 @@ spconv_status_t launch(const MapData& m, const void* x, int cin, const void* w, 
     // the fused-epilogue instantiation runs only when an epilogue op is asked for,
     // so plain layers keep the plain store
     const bool fused = epi.act != SPCONV_ACT_NONE || epi.residual != nullptr || epi.stats != nullptr;
-    auto kernel = fused ? k_subm_win<BM, KC, true> : k_subm_win<BM, KC, false>;
+    const int kind = !fused ? kEpiPlain
+                            : (epi.act == SPCONV_ACT_SILU ? kEpiSilu : (epi.act == SPCONV_ACT_GELU ? kEpiGelu : kEpiRelu));
+    auto kernel = kind == kEpiPlain  ? k_subm_win<BM, KC, kEpiPlain>
+                  : kind == kEpiRelu ? k_subm_win<BM, KC, kEpiRelu>
+                  : kind == kEpiSilu ? k_subm_win<BM, KC, kEpiSilu>
+                                     : k_subm_win<BM, KC, kEpiGelu>;
     {   // the shared-memory opt-in is per device context and instantiation
         static std::mutex attr_mu;
-        static std::vector<char> attr_done;  // bit 0: plain, bit 1: fused
+        static std::vector<char> attr_done;  // bit k: epilogue instantiation k
         std::lock_guard<std::mutex> lock(attr_mu);
         if (dev >= (int)attr_done.size()) attr_done.resize((size_t)dev + 1, 0);
-        const char bit = fused ? 2 : 1;
+        const char bit = (char)(1 << kind);
         if (!(attr_done[dev] & bit)) {
             const cudaError_t ae = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
             if (ae != cudaSuccess) {

@@ -158,7 +158,8 @@ spconv_status_t spconv_build_map_ex(const int32_t* coords, int64_t n, const int3
     if (!out_map || !extent) return fail(SPCONV_ERR_INVALID_ARG, "null extent or out_map");
     if (kernel_size != 1 && kernel_size != 3) return fail(SPCONV_ERR_INVALID_ARG, "kernel_size must be 1 or 3");
     if (n < 0 || n >= (int64_t(1) << 31)) return fail(SPCONV_ERR_INVALID_ARG, "n must be in [0, 2^31)");
-    if (flags_ & ~(uint32_t)(SPCONV_MAP_FLIP_KERNEL | SPCONV_MAP_SORTED_KEYS | SPCONV_MAP_HASH_TABLE))
+    if (flags_ & ~(uint32_t)(SPCONV_MAP_FLIP_KERNEL | SPCONV_MAP_SORTED_KEYS | SPCONV_MAP_HASH_TABLE |
+                             SPCONV_MAP_SHORT_TILES))
         return fail(SPCONV_ERR_INVALID_ARG, "unknown map flag");
     if ((flags_ & SPCONV_MAP_SORTED_KEYS) && (flags_ & SPCONV_MAP_HASH_TABLE))
         return fail(SPCONV_ERR_INVALID_ARG, "SORTED_KEYS and HASH_TABLE exclude each other");
@@ -197,7 +198,9 @@ spconv_status_t spconv_build_map_ex(const int32_t* coords, int64_t n, const int3
 
     // Every size below follows from n, so all buffers are requested up front and
     // the build needs a single synchronisation at its end.
-    d.win_rows = g_tile_rows_override > 0 ? g_tile_rows_override : spconv::choose_win_rows(n, d.num_sms);
+    d.win_rows = g_tile_rows_override > 0
+                     ? g_tile_rows_override
+                     : spconv::choose_win_rows(n, d.num_sms, (flags_ & SPCONV_MAP_SHORT_TILES) != 0);
     d.win_tiles = (n + d.win_rows - 1) / d.win_rows;
     d.npad = d.win_tiles * d.win_rows;
     const bool k3 = kernel_size == 3 && n > 0;

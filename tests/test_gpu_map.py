@@ -96,24 +96,31 @@ def test_map_errors(sp):
     _check_map(sp, coords, (16, 16, 16))
 
 
-@pytest.mark.parametrize("name", ["uniform", "shells", "large"])
+@pytest.mark.parametrize("name", ["tiny", "uniform", "shells", "batched", "large"])
 def test_tile_height_balances_the_sms(sp, name):
-    """The map's tile height is a multiple of 16 in [128, 256], and no other such
-    height gives the busiest SM fewer rows when the tiles are dealt out round-robin
-    over the device's SMs."""
+    """The map's tile height: 192 rows, or 128 with short tiles; a set too small to
+    give every SM a 192-row tile takes the multiple of 16 in [128, 192] whose busiest
+    SM gets the fewest rows when the tiles are dealt out round-robin (ties: taller)."""
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     wl = workloads.make_workload(name, 0, n_layers=1)
-    m = sp.spconv_build_map(coords_dev(wl.coords), wl.grid, 3)
-    try:
-        rows, n = m.tile_rows, wl.n
-    finally:
-        m.free()
+    heights = {}
+    for short in (False, True):
+        m = sp.spconv_build_map(coords_dev(wl.coords), wl.grid, 3, short_tiles=short)
+        try:
+            heights[short] = m.tile_rows
+        finally:
+            m.free()
+    n = wl.n
 
     def busiest(r):
         return -(-(-(-n // r)) // sms) * r
 
-    assert rows % 16 == 0 and 128 <= rows <= 256
-    assert all(busiest(rows) <= busiest(r) for r in range(128, 257, 16))
+    assert heights[True] == 128
+    if n >= sms * 192:
+        assert heights[False] == 192
+    else:
+        best = min(range(192, 127, -16), key=lambda r: (busiest(r), -r))
+        assert heights[False] == best
 
 
 # ---------------------------------------------------------------------------

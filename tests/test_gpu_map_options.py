@@ -75,7 +75,7 @@ def test_sorted_keys_errors(sp):
     # unknown flag bits are rejected by the C entry point itself
     import ctypes
     h = ctypes.c_void_p()
-    st = sp.lib.spconv_build_map_ex(None, 0, (ctypes.c_int32 * 3)(4, 4, 4), 3, 8, None, ctypes.byref(h))
+    st = sp.lib.spconv_build_map_ex(None, 0, (ctypes.c_int32 * 3)(4, 4, 4), 3, 16, None, ctypes.byref(h))
     assert st == sp.INVALID_ARG
     st = sp.lib.spconv_build_map_ex(None, 0, (ctypes.c_int32 * 3)(4, 4, 4), 3, sp.MAP_SORTED_KEYS | sp.MAP_HASH_TABLE,
                                     None, ctypes.byref(h))
