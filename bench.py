@@ -326,7 +326,7 @@ def run_per_config(sp, dev, flush, reps: int, hbm: float, tflops: float, cpu: bo
             e["map_build_ms_by_dictionary"] = {
                 "hash_table": build_ms_median(sp, coords_d, wl.grid, flush, sorted_keys=False),
                 "sorted_keys": build_ms_median(sp, coords_d, wl.grid, flush, sorted_keys=True),
-                "library_choice": "sorted_keys" if wl.n >= 1 << 20 else "hash_table"}
+                "library_choice": "hash_table"}
         if cpu:
             e["cpu_baseline"] = cpu_oracle_sample(wl, layer, target_s=1.5)
         results.append(e)

@@ -79,12 +79,11 @@ typedef enum { SPCONV_F32 = 0, SPCONV_BF16 = 1 } spconv_dtype_t;
  *   stream       stream on which the build runs.
  *   out_map      receives the handle on success; untouched on failure.
  *
- * Device work: pack (b, x, y, z) into a 64-bit key and validate it; build a
- * dictionary of the keys -- below 2^20 voxels an open-addressing hash table
- * (linear probing, 64-bit CAS, load factor <= 1/2), from 2^20 voxels on the keys
- * radix-sorted with their rows (see spconv_build_map_ex); probe the 26
- * neighbours of every voxel and write the dense map nbr[i*27 + k] = row of
- * p_i + d_k, or -1.  For kernel size 3 it then prepares
+ * Device work: pack (b, x, y, z) into a 64-bit key and validate it; insert the
+ * keys into an open-addressing hash table (linear probing, 64-bit CAS, load
+ * factor <= 1/2; spconv_build_map_ex can build radix-sorted keys instead); probe
+ * the 26 neighbours of every voxel (the first slots of three offsets loaded
+ * together) and write the dense map nbr[i*27 + k] = row of p_i + d_k, or -1.  For kernel size 3 it then prepares
  * the tensor-core forward's metadata: the rows sorted (stably, on the GPU) by the
  * Gray-code rank of their 26-bit neighbour mask, the neighbour table in that
  * order, and per tile of sorted rows the MMA jobs (see spconv_map_stats).
@@ -119,15 +118,13 @@ SPCONV_API spconv_status_t spconv_build_map(const int32_t* coords, int64_t n, co
  *                           Needs 16 + sum over axes of ceil(log2(extent)) <= 62
  *                           (SPCONV_ERR_UNSUPPORTED otherwise); never reports
  *                           SPCONV_ERR_TABLE_FULL.
- *   SPCONV_MAP_HASH_TABLE   build with the hash table whatever the size.
+ *   SPCONV_MAP_HASH_TABLE   build with the hash table (the default).
  *   SPCONV_MAP_SHORT_TILES  cut the sorted rows into 128-row tiles instead of 192:
  *                           faster for layers with 128 or more input channels
  *                           (their 16 KB gather units leave room for fewer jobs
  *                           in flight), slower for narrower ones.  Same results.
- * With neither dictionary flag the library picks one: the hash table below
- * 2^20 voxels, the sorted keys from 2^20 voxels on when the key bits fit (and
- * the hash table whenever spconv_debug_set_table_slots forces a table size).
- * Both flags together: SPCONV_ERR_INVALID_ARG.
+ * With neither dictionary flag the library builds the hash table.  Both flags
+ * together: SPCONV_ERR_INVALID_ARG.
  */
 typedef enum {
     SPCONV_MAP_DEFAULT = 0,
@@ -224,7 +221,8 @@ SPCONV_API spconv_status_t spconv_map_tile_rows(spconv_map_t map, int32_t* rows)
  *                         follow in increasing order
  *   order_dev             device int32 [tiles]: the order in which the forward's
  *                         CTAs claim the tiles, by descending estimated cost
- *                         4 * J + stream length / 16 (stable: ties by tile index)
+ *                         (4 * J + stream length / 16) / 4, integer divisions
+ *                         (stable: ties by tile index)
  * Pointers are NULL for kernel size 1 and n = 0.  The library owns them.
  * A null `map` or `stats` returns SPCONV_ERR_INVALID_ARG.
  */

@@ -206,8 +206,8 @@ def _coords_arg(coords: torch.Tensor) -> torch.Tensor:
 def spconv_build_map(coords: torch.Tensor, extent, kernel_size: int = 3, stream=None, flip_kernel: bool = False,
                      sorted_keys: bool | None = None, short_tiles: bool = False) -> SubmMap:
     """Build the neighbour map of int32 [N, 4] (b, x, y, z) CUDA coordinates.
-    ``flip_kernel`` gathers p - d_k; ``sorted_keys`` True / False forces the sorted-key
-    or the hash-table dictionary (same map); None lets the library choose by size;
+    ``flip_kernel`` gathers p - d_k; ``sorted_keys`` True builds the dictionary from
+    sorted keys instead of the hash table (same map; None and False: the hash table);
     ``short_tiles`` cuts the forward's tiles at 128 rows (faster for layers with 128
     or more input channels)."""
     _require()

@@ -79,6 +79,7 @@ __device__ __forceinline__ uint32_t gray_rank(uint32_t g) {
 }
 
 constexpr int kProbeThreads = 128;
+constexpr int kProbeBatch = 3;  // offsets whose first hash slots one thread loads together
 
 // One thread per voxel: its coordinate is read once and its 26 neighbours are
 // probed in turn.  The [rows, 27] results are staged in shared memory so the
@@ -96,30 +97,49 @@ __global__ void __launch_bounds__(kProbeThreads)
     int hits = 0;
     if (i < n) {
         const int4 c = coords[i];
-        for (int k = 0; k < kVol3; ++k) {
-            int32_t found = -1;
-            if (k == kCentre) {
-                found = (int32_t)i;
-            } else {
+        // the offsets in batches of kProbeBatch: a batch's first slots are loaded
+        // together (independent loads), then any probe whose first slot holds
+        // another key walks on alone (rare at load factor <= 1/2)
+#pragma unroll
+        for (int k0 = 0; k0 < kVol3; k0 += kProbeBatch) {
+            unsigned long long key[kProbeBatch];
+            unsigned long long slot[kProbeBatch];
+            bool inside[kProbeBatch];
+            ulonglong2 first[kProbeBatch];
+#pragma unroll
+            for (int q = 0; q < kProbeBatch; ++q) {
+                const int k = k0 + q;
                 const int x = c.y + sign * (k / 9 - 1), y = c.z + sign * ((k / 3) % 3 - 1),
                           z = c.w + sign * (k % 3 - 1);
-                if ((unsigned)x < (unsigned)ex && (unsigned)y < (unsigned)ey && (unsigned)z < (unsigned)ez) {
-                    const unsigned long long key = pack_key(c.x, x, y, z);
-                    unsigned long long slot = mix64(key) & mask;
+                inside[q] = k != kCentre && (unsigned)x < (unsigned)ex && (unsigned)y < (unsigned)ey &&
+                            (unsigned)z < (unsigned)ez;
+                key[q] = inside[q] ? pack_key(c.x, x, y, z) : kEmptyKey;
+                slot[q] = mix64(key[q]) & mask;
+                first[q] = inside[q] ? table[slot[q]] : make_ulonglong2(kEmptyKey, 0);
+            }
+#pragma unroll
+            for (int q = 0; q < kProbeBatch; ++q) {
+                const int k = k0 + q;
+                int32_t found = -1;
+                if (k == kCentre) {
+                    found = (int32_t)i;
+                } else if (inside[q]) {
+                    ulonglong2 sv = first[q];
+                    unsigned long long sl = slot[q];
                     for (unsigned long long it = 0; it <= mask; ++it) {
-                        const ulonglong2 s = table[slot];
-                        if (s.x == key) {
-                            found = (int32_t)s.y;
+                        if (sv.x == key[q]) {
+                            found = (int32_t)sv.y;
                             break;
                         }
-                        if (s.x == kEmptyKey) break;
-                        slot = (slot + 1) & mask;
+                        if (sv.x == kEmptyKey) break;
+                        sl = (sl + 1) & mask;
+                        sv = table[sl];
                     }
                 }
-                if (found >= 0) bits |= 1u << (25 - (k < kCentre ? k : k - 1));
+                if (k != kCentre && found >= 0) bits |= 1u << (25 - (k < kCentre ? k : k - 1));
+                hits += found >= 0 ? 1 : 0;
+                stage[threadIdx.x * kVol3 + k] = found;
             }
-            hits += found >= 0 ? 1 : 0;
-            stage[threadIdx.x * kVol3 + k] = found;
         }
         if (keys) keys[i] = gray_rank(bits);
     }

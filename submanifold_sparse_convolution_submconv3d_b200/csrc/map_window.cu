@@ -25,6 +25,7 @@ namespace spconv {
 namespace {
 
 constexpr int kFloorWindows = 7;  // windows of 16 columns that one MMA issue costs at least
+constexpr uint32_t kCostKeyMax = 511;  // claim-order keys take 9 bits
 
 // One thread per sorted row r (r < npad): perm[r] = the row it holds and
 // nbr_t[k * npad + r] = that row's neighbour at offset k (-1 for padding rows).
@@ -203,8 +204,10 @@ __global__ void k_win_cost(const uint32_t* __restrict__ jobs, int64_t tiles, uin
     const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (t >= tiles) return;
     const uint32_t* tj = jobs + t * kWinJobStride;
-    const uint32_t cost = 4u * tj[0] + tj[1] / 16u;
-    keys[t] = 0xFFFFu - (cost < 0xFFFFu ? cost : 0xFFFFu);  // ascending sort = descending cost
+    // cost 4 J + stream / 16 is below 2^11 (J <= 209, stream <= 27 * 256); a step of
+    // 4 (about one job) keeps the key to one 9-bit radix pass
+    const uint32_t cost = (4u * tj[0] + tj[1] / 16u) >> 2;
+    keys[t] = kCostKeyMax - (cost < kCostKeyMax ? cost : kCostKeyMax);  // ascending sort = descending cost
 }
 
 }  // namespace

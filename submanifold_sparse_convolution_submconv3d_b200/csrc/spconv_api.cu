@@ -22,7 +22,6 @@ struct spconv_map_s {
 namespace {
 
 thread_local std::string g_last_error;
-constexpr int64_t kSortedAutoMin = int64_t(1) << 20;
 int64_t g_table_slots_override = 0;
 int32_t g_tile_rows_override = 0;
 
@@ -170,12 +169,9 @@ spconv_status_t spconv_build_map_ex(const int32_t* coords, int64_t n, const int3
     const bool sorted_fits = spconv::sorted_key_bits(extent) <= 62;
     if ((flags_ & SPCONV_MAP_SORTED_KEYS) && !sorted_fits)
         return fail(SPCONV_ERR_UNSUPPORTED, "sorted-key build: 16 batch bits plus the extents' bits exceed 62");
-    // Neither dictionary forced: the hash table below kSortedAutoMin voxels, the
-    // sorted keys from there on (measured on B200: the sorted build is faster on
-    // 2.2 M voxels, the hash build on 0.2 M).
-    opts.sorted = (flags_ & SPCONV_MAP_SORTED_KEYS) != 0 ||
-                  (!(flags_ & SPCONV_MAP_HASH_TABLE) && sorted_fits && n >= kSortedAutoMin &&
-                   g_table_slots_override == 0);
+    // Neither dictionary forced: the hash table (measured on B200 with the probes
+    // batched: faster than the sorted keys on 0.2 M and 2.2 M voxels alike).
+    opts.sorted = (flags_ & SPCONV_MAP_SORTED_KEYS) != 0;
     if (n > 0 && (!coords || !aligned16(coords))) return fail(SPCONV_ERR_INVALID_ARG, "coords must be a 16-byte aligned device pointer");
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
 
@@ -257,7 +253,7 @@ spconv_status_t spconv_build_map_ex(const int32_t* coords, int64_t n, const int3
         // the row sort's buffers are free again and hold at least `tiles` entries
         if (e == cudaSuccess) e = spconv::launch_win_cost(d.win_jobs, d.win_tiles, keys[0], stream);
         int which_t = 0;
-        if (e == cudaSuccess) e = spconv::radix_sort_pairs(keys, nullptr, vals, d.win_tiles, 16, hist, &which_t, stream);
+        if (e == cudaSuccess) e = spconv::radix_sort_pairs(keys, nullptr, vals, d.win_tiles, 9, hist, &which_t, stream);
         if (e == cudaSuccess)
             e = cudaMemcpyAsync(d.win_order, vals[which_t], (size_t)d.win_tiles * sizeof(int32_t),
                                 cudaMemcpyDeviceToDevice, stream);

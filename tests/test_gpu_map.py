@@ -190,8 +190,8 @@ def _check_window_meta(sp, coords, extent):
         spans += len(k)
         cols += int(nw.sum()) * 16
     assert spans == st["spans"] and cols == st["span_cols"]
-    # claim order: a stable sort of the tiles by descending cost 4 * J + stream length // 16
-    cost = np.minimum(4 * jobs[:, 0] + jobs[:, 1] // 16, 0xFFFF)
+    # claim order: a stable sort of the tiles by descending cost (4 * J + stream length // 16) // 4
+    cost = np.minimum((4 * jobs[:, 0] + jobs[:, 1] // 16) // 4, 511)
     order = st["order"].cpu().numpy()
     assert np.array_equal(order, np.argsort(-cost, kind="stable"))
 
