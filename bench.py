@@ -94,9 +94,12 @@ def kernel_sources_sha256() -> str:
     return h.hexdigest()
 
 
-def tc_kernel_name(cin: int, cout: int) -> str:
-    """The forward kernel instantiation the library dispatches for these channels."""
+def tc_kernel_name(cin: int, cout: int, counts: dict | None = None) -> str:
+    """The forward kernel instantiation the library dispatched for these channels
+    (the map's launch counters tell the kernel-size-1 GEMM from the window kernel)."""
     bm = 128 if cout % 128 == 0 else 64
+    if counts and counts.get("tcgen05_gemm", 0) > 0:
+        return f"k_gemm1<{bm}>"
     kc = 128 if cin % 128 == 0 else 64 if cin % 64 == 0 else 32 if cin % 32 == 0 else 16
     return f"k_subm_win<{bm},{kc}>"
 
@@ -291,11 +294,12 @@ def run_per_config(sp, dev, flush, reps: int, hbm: float, tflops: float, cpu: bo
         m.check()
         layer_s = statistics.median(ms) / 1e3
         st = m.stats()
+        counts = m.launch_counts()
         e = {"config": label, "workload": name, "voxels": wl.n, "pairs": m.pairs, "cin": int(cin), "cout": int(cout),
              "kernel_size": ks, "layer_us_median": layer_s * 1e6, "layer_us_min": min(ms) * 1e3,
-             "mvox_s": wl.n / layer_s / 1e6, "kernel": tc_kernel_name(int(cin), int(cout)),
+             "mvox_s": wl.n / layer_s / 1e6, "kernel": tc_kernel_name(int(cin), int(cout), counts),
              "roofline": roofline(wl.n, m.pairs, int(cin), int(cout), int(kvol), layer_s, hbm, tflops),
-             "rows_per_tile": st["rows_per_tile"], "tiles": st["tiles"], "launch_counts": m.launch_counts()}
+             "rows_per_tile": st["rows_per_tile"], "tiles": st["tiles"], "launch_counts": counts}
         if ks == 3:
             e["spans"] = st["spans"]
             e["issued_column_efficiency"] = issued_column_efficiency(m.pairs, st["tiles"] * st["rows_per_tile"],
@@ -446,21 +450,22 @@ def run_resample_chain(sp, dev, flush, reps: int = 5) -> dict:
 def run_profile_mode(args) -> None:
     """A small fixed run for ncu captures (committed, so profile summaries can name
     their command): --profile-layer NAME runs the map build and three launches of
-    the workload's first layer; --profile-build NAME:DICT runs three map builds with
-    the dictionary DICT (hash, sorted or auto)."""
+    the workload's first layer (NAME:I: its layer I); --profile-build NAME:DICT runs
+    three map builds with the dictionary DICT (hash, sorted or auto)."""
     import torch
 
     import submanifold_sparse_convolution_submconv3d_b200 as sp
     dev = torch.device("cuda", 0)
     if args.profile_layer:
-        wl = workloads.make_workload(args.profile_layer, 0, n_layers=1)
+        name, _, li = args.profile_layer.partition(":")
+        wl = workloads.make_workload(name, 0, n_layers=1)
+        layer = wl.layers[int(li or 0)]
         # the map as the benchmark builds it: short tiles for 128+-channel layers
-        short = int(wl.layers[0].w.shape[1]) >= 128
-        m = sp.spconv_build_map(torch.from_numpy(wl.coords).to(dev), wl.grid, wl.layers[0].kernel_size,
-                                short_tiles=short)
+        short = int(layer.w.shape[1]) >= 128
+        m = sp.spconv_build_map(torch.from_numpy(wl.coords).to(dev), wl.grid, layer.kernel_size, short_tiles=short)
         x = torch.from_numpy(wl.x).to(dev, torch.bfloat16)
-        w = torch.from_numpy(wl.layers[0].w).to(dev, torch.bfloat16)
-        b = torch.from_numpy(wl.layers[0].bias).to(dev, torch.bfloat16)
+        w = torch.from_numpy(layer.w).to(dev, torch.bfloat16)
+        b = torch.from_numpy(layer.bias).to(dev, torch.bfloat16)
         out = torch.empty((wl.n, w.shape[2]), dtype=torch.bfloat16, device=dev)
         for _ in range(3):
             sp.spconv_subm_forward(m, x, w, b, out=out)
@@ -673,7 +678,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true")
-    ap.add_argument("--profile-layer", default=None, help="workload: map build + 3 launches of its first layer (ncu)")
+    ap.add_argument("--profile-layer", default=None, help="workload[:layer]: map build + 3 launches of the layer (ncu)")
     ap.add_argument("--profile-build", default=None, help="workload:hash|sorted|auto: 3 map builds (ncu)")
     args = ap.parse_args()
     if args.profile_layer or args.profile_build:

@@ -158,9 +158,12 @@ SPCONV_API spconv_status_t spconv_build_map_ex(const int32_t* coords, int64_t n,
  *   stream  stream on which the layer runs.
  *
  * Accumulation is fp32 in every mode; the bf16 result is rounded to nearest even.
- * bf16 with cout a multiple of 64 runs on the tensor-core (tcgen05) kernel; fp32,
- * and bf16 with other channel counts, on a CUDA-core kernel.  The choice depends
- * on dtype and cout alone; spconv_map_launch_counts reports which kernel ran.
+ * bf16 with cout a multiple of 64 runs on the tensor cores (tcgen05): a map of
+ * kernel size 1 with cin a multiple of 64 (cin <= 704 when cout % 128 == 0, else
+ * cin <= 1472) and n >= 128 on a weight-stationary GEMM, every other such layer
+ * on the window kernel; fp32, and bf16 with other channel counts, on a CUDA-core
+ * kernel.  The choice depends on dtype, the kernel size, n and the channel
+ * counts alone; spconv_map_launch_counts reports which kernel ran.
  * The layer runs on the current CUDA device, which must be the device the map
  * was built on (otherwise SPCONV_ERR_INVALID_ARG).
  * The call only validates on the host and launches; it never synchronises.
@@ -255,8 +258,9 @@ SPCONV_API const char* spconv_last_error(void);
  *   SPCONV_ALGO_AUTO     what spconv_subm_forward uses: the tcgen05 kernel for bf16
  *                        when cout % 64 == 0, the CUDA-core kernel otherwise.
  *   SPCONV_ALGO_SIMT     CUDA-core FMA kernel, any channel count, fp32 or bf16.
- *   SPCONV_ALGO_TCGEN05  tcgen05 tensor-core kernel (bf16, cin % 16 == 0,
- *                        cout % 64 == 0; SPCONV_ERR_UNSUPPORTED otherwise).
+ *   SPCONV_ALGO_TCGEN05  the tcgen05 tensor-core kernels (bf16, cin % 16 == 0,
+ *                        cout % 64 == 0; SPCONV_ERR_UNSUPPORTED otherwise): the
+ *                        same GEMM-or-window choice as AUTO.
  * Same arguments, ownership and errors as spconv_subm_forward.
  */
 typedef enum { SPCONV_ALGO_AUTO = 0, SPCONV_ALGO_SIMT = 1, SPCONV_ALGO_TCGEN05 = 2 } spconv_algo_t;
@@ -309,8 +313,9 @@ SPCONV_API spconv_status_t spconv_subm_forward_ex(spconv_map_t map, spconv_dtype
  */
 typedef enum {
     SPCONV_KERNEL_SIMT = 0,     /* CUDA-core FMA kernel: fp32, and bf16 shapes no tensor-core kernel takes */
-    SPCONV_KERNEL_TCGEN05 = 1,  /* tcgen05 tensor-core kernel */
-    SPCONV_KERNEL_KINDS = 2
+    SPCONV_KERNEL_TCGEN05 = 1,  /* tcgen05 tensor-core window kernel (gathered rows) */
+    SPCONV_KERNEL_TCGEN05_GEMM = 2, /* tcgen05 weight-stationary GEMM: kernel size 1, cin % 64 == 0, n >= 128 */
+    SPCONV_KERNEL_KINDS = 3
 } spconv_kernel_t;
 
 /*
@@ -342,7 +347,9 @@ SPCONV_API spconv_status_t spconv_debug_set_tile_rows(int32_t rows);
  * Test hook: force the tensor-core forward's ring depths for later launches in
  * this process: a_slots weight tiles in [2, 8] and b_units units of 64 gathered
  * rows in [4, 32]; (0, 0) restores the automatic choice.  A launch whose forced
- * depths do not fit shared memory returns SPCONV_ERR_UNSUPPORTED.  Lets tests
+ * depths do not fit shared memory returns SPCONV_ERR_UNSUPPORTED.  The
+ * kernel-size-1 GEMM takes a_slots as its count of x stages (fewer if they do
+ * not fit).  Lets tests
  * drive shallow rings (frequent wrap-around) and the benchmark sweep depths.
  * Other values: SPCONV_ERR_INVALID_ARG.
  */

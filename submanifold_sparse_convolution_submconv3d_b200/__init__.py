@@ -29,7 +29,7 @@ OK, INVALID_ARG, UNSUPPORTED, COORD_RANGE, DUPLICATE, TABLE_FULL, OOM, CUDA_ERRO
 MAP_DEFAULT, MAP_FLIP_KERNEL, MAP_SORTED_KEYS, MAP_HASH_TABLE, MAP_SHORT_TILES = 0, 1, 2, 4, 8
 ALGO_AUTO, ALGO_SIMT, ALGO_TCGEN05 = 0, 1, 2
 KERNEL_SIMT, KERNEL_TCGEN05 = 0, 1
-KERNEL_NAMES = ("simt", "tcgen05")
+KERNEL_NAMES = ("simt", "tcgen05", "tcgen05_gemm")
 _DTYPES = {torch.float32: 0, torch.bfloat16: 1}
 
 EXPORTED = ("spconv_build_map", "spconv_subm_forward", "spconv_free", "spconv_map_info", "spconv_map_check",

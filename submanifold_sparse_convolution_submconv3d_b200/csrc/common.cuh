@@ -192,6 +192,17 @@ cudaError_t launch_forward_simt(const MapData& m, spconv_dtype_t dtype, const vo
 // units of later launches (0, 0: automatic).
 void set_forced_ring_depths(int sa, int ub);
 
+// Kernel size 1 as a weight-stationary tcgen05 GEMM (forward_gemm1.cu): bf16,
+// cin % 64 == 0 with the weight slice and two x stages in shared memory (cin <=
+// 704 when cout % 128 == 0, else 1472), cout % 64 == 0, n >= 128.  Returns SPCONV_OK,
+// SPCONV_ERR_UNSUPPORTED (shape not handled) or SPCONV_ERR_CUDA.
+spconv_status_t launch_forward_gemm1(const MapData& m, const void* x, int cin, const void* w, const void* bias,
+                                     void* out, int cout, const Epilogue& epi, cudaStream_t stream,
+                                     cudaError_t* cuda_err);
+
+// Test hook of the kernel-size-1 GEMM: x stages of later launches (0: as many as fit).
+void set_forced_gemm1_stages(int stages);
+
 // Returns SPCONV_OK, SPCONV_ERR_UNSUPPORTED (shape not handled) or SPCONV_ERR_CUDA.
 spconv_status_t launch_forward_tcgen05(const MapData& m, const void* x, int cin, const void* w,
                                        const void* bias, void* out, int cout, const Epilogue& epi,

@@ -56,11 +56,19 @@
 
 #include "common.cuh"
 #include "sm100.cuh"
+#include "tc_common.cuh"
 
 namespace spconv {
 namespace {
 
 using namespace sm100;
+using tc::kEpiGelu;
+using tc::kEpiPlain;
+using tc::kEpiRelu;
+using tc::kEpiSilu;
+using tc::kWaitTimeoutNs;
+using tc::wait_bar;
+using tc::warp_wait_bar;
 
 constexpr int kWarpMma = 0, kWarpTma = 1, kWarpGather0 = 2, kGatherWarps = 4, kEpiWarps = 8;
 constexpr int kWarpEpi0 = kWarpGather0 + kGatherWarps;
@@ -72,10 +80,6 @@ constexpr int kThreads = 32 * (kWarpPrep + 1);          // 480
 constexpr int kCmdSlots = 16;
 constexpr uint32_t kCmdRelA = 1, kCmdInit = 2, kCmdFirst = 4, kCmdTileEnd = 8, kCmdExit = 16;
 constexpr int kEpiGroups = kEpiWarps / 4;  // epilogue warps per TMEM lane quarter
-// Kernel instantiations by epilogue: the plain store, and the fused epilogue with
-// ReLU or none (chosen at run time), SiLU or GELU, so no instantiation carries the
-// code of the activations it does not run.
-constexpr int kEpiPlain = 0, kEpiRelu = 1, kEpiSilu = 2, kEpiGelu = 3;
 static_assert(kEpiWarps % 4 == 0 && kWinMaxRows / 32 % kEpiGroups == 0, "whole lane quarters, whole chunks");
 constexpr int kAccBufs = 2;
 constexpr int kIdxBufs = 2;
@@ -90,7 +94,6 @@ static_assert(kAccBufs * kAccCols <= kTmemCols, "accumulators must fit TMEM");
 constexpr int kUnitRows = 64;          // rows of one B-ring unit
 constexpr int kMaxUnits = 32;          // the per-unit phase bits live in one 32-bit word
 constexpr int kMaxASlots = 8;
-constexpr uint64_t kWaitTimeoutNs = 4000000000ull;
 constexpr int kMaxSmem = 232448;       // 227 KB opt-in limit per CTA on sm_100
 constexpr int kMinSmem = 120 * 1024;   // keeps one CTA per SM: each CTA allocates all 512 TMEM columns
 
@@ -166,38 +169,6 @@ struct WinParams {
 // less on the 512-channel one without a pause).  The epilogue waits for a whole
 // tile of MMAs and backs off up to 2 us.
 constexpr uint32_t kSleepMma = 0, kSleepProducer = 0, kSleepEpilogue = 2048;
-
-template <uint32_t kMaxSleepNs>
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag, unsigned int* err) {
-    if (mbar_try_wait(bar, parity)) return true;
-    uint64_t t0 = 0;
-    uint32_t pause = 32;
-    for (uint32_t i = 1;; ++i) {
-        if constexpr (kMaxSleepNs > 0) {
-            __nanosleep(pause);
-            pause = pause < kMaxSleepNs ? 2 * pause : pause;
-        }
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 15u) != 0) continue;  // the timer and the abort flag every few polls
-        if (*abort_flag) return false;
-        const uint64_t now = globaltimer_ns();
-        if (t0 == 0) {
-            t0 = now;
-        } else if (now - t0 > kWaitTimeoutNs) {
-            *abort_flag = 1;
-            atomicOr(err, kFwdErrTimeout);
-            return false;
-        }
-    }
-}
-
-template <uint32_t kMaxSleepNs>
-__device__ __forceinline__ bool warp_wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                              unsigned int* err) {
-    int ok = 1;
-    if ((threadIdx.x & 31) == 0) ok = wait_bar<kMaxSleepNs>(bar, parity, abort_flag, err) ? 1 : 0;
-    return __shfl_sync(0xffffffffu, ok, 0) != 0;
-}
 
 // B-ring units of the next (job, chunk): ceil(N / 64) consecutive units, starting
 // over at unit 0 when they would run past the end.  Every role runs this on the
@@ -676,9 +647,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int half = (warp - kWarpEpi0) >> 2;  // this warp's group within its lane quarter
         const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
         __nv_bfloat16* stg = stage + (warp - kWarpEpi0) * L::kStageRows * L::kChPerWarp;
-        constexpr int kVecPerRow = L::kChPerWarp * 2 / 16;
         constexpr int kChunksPerWarp = kWinMaxRows / 32 / kEpiGroups;  // this warp's 32-column chunks of a tile
         const bool lane_ok = lane < L::kChPerWarp;
+        const tc::EpiOut eo{p.out, p.residual, p.cout, p.act};
         for (int i = 0; !aborted; ++i) {
             const int s = i % kTileSlots;
             const uint8_t* slot = tile_ring + s * kSlotBytes;
@@ -726,71 +697,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     float v[32];
                     tmem_ld_x32(tmem + lane_base + (uint32_t)buf * kAccCols + (uint32_t)(cc * 32), v);
                     tmem_wait_ld();
-#pragma unroll
-                    for (int hp = 0; hp < 32 / L::kStageRows; ++hp) {
-                        if constexpr (kEpi == kEpiPlain) {
-                            if (lane_ok) {
-#pragma unroll
-                                for (int e = 0; e < L::kStageRows; ++e)
-                                    stg[e * L::kChPerWarp + lane] =
-                                        __float2bfloat16_rn(v[hp * L::kStageRows + e] + bv);
-                            }
-                        } else {
-                            // fused epilogue: act(conv + bias) (+ residual) in fp32, then the
-                            // rounded value is stored and counted in the statistics
-                            const int col0 = cc * 32 + hp * L::kStageRows;  // tile column of row e = col0 + e
-                            float rv[L::kStageRows];  // residual elements (0 when there is none)
-                            if (p.residual) {
-                                // the output rows of these columns, then their residual
-                                // elements, loaded together (a missing row reads row 0)
-                                int ro[L::kStageRows];
-#pragma unroll
-                                for (int e = 0; e < L::kStageRows; ++e)
-                                    ro[e] = __shfl_sync(0xffffffffu, orow[c4], hp * L::kStageRows + e);
-#pragma unroll
-                                for (int e = 0; e < L::kStageRows; ++e)
-                                    rv[e] = lane_ok ? __bfloat162float(p.residual[(int64_t)(ro[e] > 0 ? ro[e] : 0) *
-                                                                                      p.cout + ch_base + lane])
-                                                    : 0.0f;
-                            } else {
-#pragma unroll
-                                for (int e = 0; e < L::kStageRows; ++e) rv[e] = 0.0f;
-                            }
-                            if (lane_ok) {
-#pragma unroll
-                                for (int e = 0; e < L::kStageRows; ++e) {
-                                    float y = v[hp * L::kStageRows + e] + bv;
-                                    if constexpr (kEpi == kEpiRelu) {
-                                        if (p.act == SPCONV_ACT_RELU) y = fmaxf(y, 0.0f);
-                                    } else if constexpr (kEpi == kEpiSilu) {
-                                        // fast exponential and division: their error is far below the
-                                        // bf16 rounding of out (a huge denominator gives -0 for y << 0)
-                                        y = __fdividef(y, 1.0f + __expf(-y));
-                                    } else {
-                                        y = epi_act(SPCONV_ACT_GELU, y);
-                                    }
-                                    const __nv_bfloat16 q = __float2bfloat16_rn(y + rv[e]);
-                                    stg[e * L::kChPerWarp + lane] = q;
-                                    if (col0 + e < t_eff) {
-                                        const float f = __bfloat162float(q);
-                                        s1 += f;
-                                        s2 += f * f;
-                                    }
-                                }
-                            }
-                        }
-                        __syncwarp();
-#pragma unroll
-                        for (int e = lane; e < L::kStageRows * kVecPerRow; e += 32) {
-                            const int row = e / kVecPerRow, vq = e % kVecPerRow;
-                            const int o = __shfl_sync(0xffffffffu, orow[c4], hp * L::kStageRows + row);
-                            if (o >= 0) {
-                                const int4 val = *reinterpret_cast<const int4*>(stg + row * L::kChPerWarp + vq * 8);
-                                *reinterpret_cast<int4*>(p.out + (int64_t)o * p.cout + ch_base + vq * 8) = val;
-                            }
-                        }
-                        __syncwarp();
-                    }
+                    tc::store_chunk<kEpi, L::kChPerWarp, L::kStageRows>(v, orow[c4], lane, lane_ok, bv, ch_base,
+                                                                        cc * 32, t_eff, eo, stg, s1, s2);
                 }
             }
             if constexpr (kEpi != kEpiPlain) {
@@ -813,23 +721,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
-}
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* f = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(f);
-    });
-    return fn;
 }
 
 int g_force_sa = 0, g_force_ub = 0;  // test hook: ring depths (0 = automatic)
@@ -864,7 +755,7 @@ template <int BM, int KC>
 spconv_status_t launch(const MapData& m, const void* x, int cin, const void* w, const void* bias, void* out,
                        int cout, const Epilogue& epi, cudaStream_t stream, cudaError_t* ce) {
     using L = WinLayout<BM, KC>;
-    EncodeTiledFn enc = encode_fn();
+    tc::EncodeTiledFn enc = tc::encode_fn();
     if (!enc) {
         *ce = cudaErrorSymbolNotFound;
         return SPCONV_ERR_CUDA;
@@ -918,9 +809,7 @@ spconv_status_t launch(const MapData& m, const void* x, int cin, const void* w, 
     }
     // the fused-epilogue instantiation runs only when an epilogue op is asked for,
     // so plain layers keep the plain store
-    const bool fused = epi.act != SPCONV_ACT_NONE || epi.residual != nullptr || epi.stats != nullptr;
-    const int kind = !fused ? kEpiPlain
-                            : (epi.act == SPCONV_ACT_SILU ? kEpiSilu : (epi.act == SPCONV_ACT_GELU ? kEpiGelu : kEpiRelu));
+    const int kind = tc::epi_kind(epi);
     auto kernel = kind == kEpiPlain  ? k_subm_win<BM, KC, kEpiPlain>
                   : kind == kEpiRelu ? k_subm_win<BM, KC, kEpiRelu>
                   : kind == kEpiSilu ? k_subm_win<BM, KC, kEpiSilu>

@@ -130,6 +130,7 @@ spconv_status_t spconv_debug_set_ring_depths(int32_t a_slots, int32_t b_units) {
     if (!auto_ && (a_slots < 2 || a_slots > 8 || b_units < 4 || b_units > 32))
         return fail(SPCONV_ERR_INVALID_ARG, "a_slots must be in [2, 8] and b_units in [4, 32], or both 0");
     spconv::set_forced_ring_depths(a_slots, b_units);
+    spconv::set_forced_gemm1_stages(a_slots);
     return SPCONV_OK;
 }
 
@@ -384,12 +385,22 @@ spconv_status_t spconv_subm_forward_ex(spconv_map_t map, spconv_dtype_t dtype, c
     }
     if (algo == SPCONV_ALGO_TCGEN05 && dtype != SPCONV_BF16)
         return fail(SPCONV_ERR_UNSUPPORTED, "the tcgen05 kernel is bf16 only");
-    // AUTO: bf16 with cout % 64 == 0 runs on the tensor cores; fp32 and other bf16
-    // shapes on the CUDA-core kernel.  The choice depends on the shape alone, and
-    // the map's launch counters record it.
+    // AUTO: bf16 with cout % 64 == 0 runs on the tensor cores (kernel size 1 on
+    // the weight-stationary GEMM when it takes the shape, else on the window
+    // kernel); fp32 and other bf16 shapes on the CUDA-core kernel.  The choice
+    // depends on the shape alone, and the map's launch counters record it.
     const bool tc_shape = dtype == SPCONV_BF16 && cout % 64 == 0;
     if (algo == SPCONV_ALGO_TCGEN05 || (algo == SPCONV_ALGO_AUTO && tc_shape)) {
         cudaError_t ce = cudaSuccess;
+        if (map->d.kernel_size == 1) {
+            const spconv_status_t g =
+                spconv::launch_forward_gemm1(map->d, x, cin, w, bias, out, cout, epi, stream, &ce);
+            if (g == SPCONV_ERR_CUDA) return fail_cuda(ce, "tcgen05 GEMM forward");
+            if (g == SPCONV_OK) {
+                map->launches[SPCONV_KERNEL_TCGEN05_GEMM].fetch_add(1);
+                return SPCONV_OK;
+            }
+        }
         const spconv_status_t s = spconv::launch_forward_tcgen05(map->d, x, cin, w, bias, out, cout, epi, stream, &ce);
         if (s == SPCONV_ERR_CUDA) return fail_cuda(ce, "tcgen05 forward");
         if (s != SPCONV_OK)

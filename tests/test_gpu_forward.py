@@ -256,12 +256,16 @@ def test_repeat_calls_identical(sp):
 
 @pytest.mark.parametrize("name", ["tiny", "uniform", "shells", "batched", "large"])
 def test_auto_kernel_choice_on_workloads(sp, name):
-    """AUTO runs every bf16 layer of the five workloads on the tensor cores (and the
-    fp32 tiny layers on the CUDA-core kernel); the map's launch counters show it."""
+    """AUTO runs every bf16 layer of the five workloads on the tensor cores (kernel
+    size 1 with 64-channel multiples on the GEMM kernel, the rest on the window
+    kernel) and the fp32 tiny layers on the CUDA-core kernel; the map's launch
+    counters show it."""
     wl = workloads.make_workload(name, 0, n_layers=1)
-    expected = "simt" if wl.dtype == "f32" else "tcgen05"
     x = to_dev(wl.x, wl.dtype)
     for layer in wl.layers:
+        cin = layer.w.shape[1]
+        expected = ("simt" if wl.dtype == "f32" else
+                    "tcgen05_gemm" if layer.kernel_size == 1 and cin % 64 == 0 and wl.n >= 128 else "tcgen05")
         m = sp.spconv_build_map(coords_dev(wl.coords), wl.grid, layer.kernel_size)
         try:
             sp.spconv_subm_forward(m, x, to_dev(layer.w, wl.dtype), to_dev(layer.bias, wl.dtype))
