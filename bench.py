@@ -76,7 +76,7 @@ PROFILED_TRAFFIC = {
     "bytes": 87197440,
     "sources_sha256": "55a9878c4a5407096453b1894d2de3d7af41e0f3d0b763b8fb8460b193fa0fca",
 }
-KERNEL_SOURCES = ("forward_win.cu", "sm100.cuh", "common.cuh")
+KERNEL_SOURCES = ("forward_win.cu", "tc_common.cuh", "sm100.cuh", "common.cuh")
 
 
 def kernel_sources_sha256() -> str:
