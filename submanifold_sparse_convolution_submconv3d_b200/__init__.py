@@ -28,7 +28,7 @@ LIB_PATH = os.path.join(_HERE, "libspconv_b200.so")
 OK, INVALID_ARG, UNSUPPORTED, COORD_RANGE, DUPLICATE, TABLE_FULL, OOM, CUDA_ERROR, TIMEOUT = range(9)
 MAP_DEFAULT, MAP_FLIP_KERNEL, MAP_SORTED_KEYS, MAP_HASH_TABLE, MAP_SHORT_TILES = 0, 1, 2, 4, 8
 ALGO_AUTO, ALGO_SIMT, ALGO_TCGEN05 = 0, 1, 2
-KERNEL_SIMT, KERNEL_TCGEN05 = 0, 1
+KERNEL_SIMT, KERNEL_TCGEN05, KERNEL_TCGEN05_GEMM = 0, 1, 2
 KERNEL_NAMES = ("simt", "tcgen05", "tcgen05_gemm")
 _DTYPES = {torch.float32: 0, torch.bfloat16: 1}
 
@@ -449,4 +449,5 @@ __all__ = ["OK", "INVALID_ARG", "UNSUPPORTED", "COORD_RANGE", "DUPLICATE", "TABL
            "spconv_downsample_amax", "spconv_upsample", "spconv_subdivide", "MAP_DEFAULT", "MAP_FLIP_KERNEL",
            "MAP_SORTED_KEYS", "MAP_HASH_TABLE", "MAP_SHORT_TILES", "ACTIVATIONS",
            "LIB_PATH", "EXPORTED",
-           "ALGO_AUTO", "ALGO_SIMT", "ALGO_TCGEN05", "KERNEL_SIMT", "KERNEL_TCGEN05", "KERNEL_NAMES"]
+           "ALGO_AUTO", "ALGO_SIMT", "ALGO_TCGEN05", "KERNEL_SIMT", "KERNEL_TCGEN05", "KERNEL_TCGEN05_GEMM",
+           "KERNEL_NAMES"]

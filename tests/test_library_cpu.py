@@ -31,6 +31,32 @@ def test_header_declares_the_boundary():
     assert len(syms) >= 8
 
 
+def _header_enum(prefix):
+    """{name: value} of the header's enumerators starting with prefix."""
+    text = open(HEADER).read()
+    return {m.group(1): int(m.group(2)) for m in re.finditer(r"\b(" + prefix + r"\w+)\s*=\s*(\d+)", text)}
+
+
+def test_binding_constants_match_the_header(pkg):
+    """The binding's copies of the header's enumerators (map flags, algorithms,
+    activations, kernel families) carry the header's values."""
+    maps = _header_enum("SPCONV_MAP_")
+    assert (pkg.MAP_DEFAULT, pkg.MAP_FLIP_KERNEL, pkg.MAP_SORTED_KEYS, pkg.MAP_HASH_TABLE, pkg.MAP_SHORT_TILES) == (
+        maps["SPCONV_MAP_DEFAULT"], maps["SPCONV_MAP_FLIP_KERNEL"], maps["SPCONV_MAP_SORTED_KEYS"],
+        maps["SPCONV_MAP_HASH_TABLE"], maps["SPCONV_MAP_SHORT_TILES"])
+    algos = _header_enum("SPCONV_ALGO_")
+    assert (pkg.ALGO_AUTO, pkg.ALGO_SIMT, pkg.ALGO_TCGEN05) == (
+        algos["SPCONV_ALGO_AUTO"], algos["SPCONV_ALGO_SIMT"], algos["SPCONV_ALGO_TCGEN05"])
+    acts = _header_enum("SPCONV_ACT_")
+    for name in ("none", "relu", "silu", "gelu"):
+        assert pkg.ACTIVATIONS[name] == acts["SPCONV_ACT_" + name.upper()]
+    kinds = _header_enum("SPCONV_KERNEL_")
+    assert len(pkg.KERNEL_NAMES) == kinds["SPCONV_KERNEL_KINDS"]
+    assert (pkg.KERNEL_SIMT, pkg.KERNEL_TCGEN05, pkg.KERNEL_TCGEN05_GEMM) == (
+        kinds["SPCONV_KERNEL_SIMT"], kinds["SPCONV_KERNEL_TCGEN05"], kinds["SPCONV_KERNEL_TCGEN05_GEMM"])
+    assert pkg.KERNEL_NAMES[pkg.KERNEL_TCGEN05_GEMM] == "tcgen05_gemm"
+
+
 def test_library_exports_every_declared_symbol(pkg):
     lib = ctypes.CDLL(pkg.LIB_PATH)
     for name in _declared_symbols():
