@@ -92,3 +92,7 @@ def test_tc_kernel_name_follows_the_dispatch():
     assert bench.tc_kernel_name(64, 64) == "k_subm_win<64,64>"
     assert bench.tc_kernel_name(48, 192) == "k_subm_win<64,16>"
     assert bench.tc_kernel_name(32, 256) == "k_subm_win<128,32>"
+    # the map's launch counters name the kernel-size-1 GEMM when it ran
+    assert bench.tc_kernel_name(512, 512, {"simt": 0, "tcgen05": 0, "tcgen05_gemm": 1}) == "k_gemm1<128>"
+    assert bench.tc_kernel_name(64, 192, {"simt": 0, "tcgen05": 0, "tcgen05_gemm": 1}) == "k_gemm1<64>"
+    assert bench.tc_kernel_name(48, 128, {"simt": 0, "tcgen05": 1, "tcgen05_gemm": 0}) == "k_subm_win<128,16>"
