@@ -255,8 +255,9 @@ SPCONV_API const char* spconv_last_error(void);
 
 /*
  * Forward with an explicit kernel family, for cross-checks:
- *   SPCONV_ALGO_AUTO     what spconv_subm_forward uses: the tcgen05 kernel for bf16
- *                        when cout % 64 == 0, the CUDA-core kernel otherwise.
+ *   SPCONV_ALGO_AUTO     what spconv_subm_forward uses: the tcgen05 kernels for
+ *                        bf16 when cout % 64 == 0 (the GEMM or the window kernel,
+ *                        as described there), the CUDA-core kernel otherwise.
  *   SPCONV_ALGO_SIMT     CUDA-core FMA kernel, any channel count, fp32 or bf16.
  *   SPCONV_ALGO_TCGEN05  the tcgen05 tensor-core kernels (bf16, cin % 16 == 0,
  *                        cout % 64 == 0; SPCONV_ERR_UNSUPPORTED otherwise): the
@@ -349,8 +350,8 @@ SPCONV_API spconv_status_t spconv_debug_set_tile_rows(int32_t rows);
  * rows in [4, 32]; (0, 0) restores the automatic choice.  A launch whose forced
  * depths do not fit shared memory returns SPCONV_ERR_UNSUPPORTED.  The
  * kernel-size-1 GEMM takes a_slots as its count of x stages (fewer if they do
- * not fit).  Lets tests
- * drive shallow rings (frequent wrap-around) and the benchmark sweep depths.
+ * not fit).  Lets tests drive shallow rings (frequent wrap-around) and the
+ * benchmark sweep depths.
  * Other values: SPCONV_ERR_INVALID_ARG.
  */
 SPCONV_API spconv_status_t spconv_debug_set_ring_depths(int32_t a_slots, int32_t b_units);
